@@ -1,0 +1,454 @@
+"""Benchmark of the paged-KV attention hot path on B200.
+
+Default workload: one decode step at batch 512 with prefix sharing (lognormal context
+lengths, median 1024, clipped to [16, 4096]; half the sequences share a 1024-token prefix
+held in 4 physical blocks; 16 query / 8 KV heads, head_dim 128, block size 256, bf16).
+A step is store_kvcache of the 512 new tokens followed by paged decode attention.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl nvpa|reference]
+                    [--workload NAME]
+
+Prints one JSON line.  `value` is the achieved HBM bandwidth of the whole step in GB/s,
+counting each unique cached K/V row once (plus q, out, the new rows and the index
+arrays); `seq_steps_per_s` is batch / step time.  Under torchrun (N > 1) every rank runs
+its own batch (weak scaling, no collective on the data path); the time is the maximum
+over ranks.  `--impl reference` times the CPU oracle on a bounded sample instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "paged decode attn: achieved HBM GB/s (% of peak), seq-steps/s at batch 512"
+DEFAULT_WORKLOAD = "decode_b512_shared_prefix"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+# ----------------------------------------------------------------------------------
+# algorithmic work (bytes / flops) of a step, from the workload's metadata
+# ----------------------------------------------------------------------------------
+
+def decode_step_bytes(step) -> dict:
+    """Algorithmic HBM bytes of one decode step (store + attention).
+
+    Each physical (block, row) that holds a live token is read once per KV head for K and
+    for V, even when several sequences share it; q is read and out written once; the
+    store reads the new K/V rows and writes them; index arrays are read once.
+    """
+    bs, hkv, d = step.block_size, step.num_kv_heads, step.head_dim
+    used = {}
+    for b in range(step.batch):
+        L = int(step.context_lens[b])
+        for j in range((L + bs - 1) // bs):
+            blk = int(step.block_tables[b, j])
+            used[blk] = max(used.get(blk, 0), min(bs, L - j * bs))
+    unique_rows = sum(used.values())
+    kv = unique_rows * hkv * d * 2 * 2
+    logical_kv = int(step.context_lens.sum()) * hkv * d * 2 * 2
+    qo = 2 * step.batch * step.num_q_heads * d * 2
+    n_real = int((step.slot_mapping >= 0).sum())
+    store = 2 * n_real * hkv * d * 2 * 2 + step.num_tokens * 4
+    tables = sum((int(L) + bs - 1) // bs for L in step.context_lens) * 4 + step.batch * 4
+    return dict(kv_unique=kv, kv_logical=logical_kv, attention=kv + qo + tables,
+                store=store, step=kv + qo + tables + store)
+
+
+def prefill_step_work(step) -> dict:
+    d, hq, hkv = step.head_dim, step.num_q_heads, step.num_kv_heads
+    flops = 0
+    for i in range(step.batch):
+        lq = int(step.cu_seqlens_q[i + 1] - step.cu_seqlens_q[i])
+        lk = int(step.cu_seqlens_k[i + 1] - step.cu_seqlens_k[i])
+        # query r sees lk - lq + r + 1 keys; QK^T and PV are 2*d flops per (query, key) each
+        flops += 4 * d * hq * (lq * (lk - lq) + lq * (lq + 1) // 2)
+    store = 2 * step.total_q * hkv * d * 2 * 2 + step.total_q * 4
+    return dict(flops=flops, store=store)
+
+
+# ----------------------------------------------------------------------------------
+# environment helpers
+# ----------------------------------------------------------------------------------
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16_tflops=float(p["bf16_tflops"]),
+                    bf16_tflops_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm_gbs=FALLBACK_HBM_GBS, bf16_tflops=FALLBACK_BF16_TFLOPS,
+                    bf16_tflops_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples taken while the timed region runs."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={CLOCK_QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self) -> dict:
+        if self.proc is None or not os.path.exists(self.path):
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvidia-smi unavailable"])
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return dict(sm_mhz=None, sm_max_mhz=smax, reasons=["no samples"])
+        busy = sorted(sm)[len(sm) // 4:] or sm   # drop idle samples at the edges
+        return dict(sm_mhz=float(np.median(busy)), sm_max_mhz=smax, reasons=sorted(reasons),
+                    samples=len(sm))
+
+
+def profile_traffic(kernel_tag: str, source_files) -> float | None:
+    """DRAM bytes per launch recorded in profiles/ for this kernel, if the kernel's source
+    is unchanged since the capture (the summary stores a hash of its sources)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel_tag}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"source_sha256:\s*([0-9a-f]{16,64})", text)
+    if not m or not h:
+        return None
+    digest = hashlib.sha256()
+    for f in source_files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            digest.update(fh.read())
+    if not digest.hexdigest().startswith(h.group(1)):
+        return None
+    return float(m.group(1))
+
+
+DECODE_SOURCES = ["paged_kv_cache_422_b200/csrc/paged_attention.cu",
+                  "paged_kv_cache_422_b200/csrc/attn_warp.cuh",
+                  "paged_kv_cache_422_b200/csrc/common.cuh"]
+
+
+def source_sha(files) -> str:
+    digest = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            digest.update(fh.read())
+    return digest.hexdigest()
+
+
+# ----------------------------------------------------------------------------------
+# distributed plumbing (also exercised by the gloo tests)
+# ----------------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Maximum of a per-rank float over the process group (identity with one process)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------------------------
+# CPU oracle (reference arm and cpu_baseline)
+# ----------------------------------------------------------------------------------
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_decode_sample(step, seqs):
+    """Run the CPU oracle's decode over a sample of sequences; returns (seconds, bytes)."""
+    import oracle
+    t0 = time.perf_counter()
+    oracle.paged_decode_attention(step.q[seqs], step._ora_k, step._ora_v, step.block_tables[seqs],
+                                  step.context_lens[seqs], step.scale)
+    dt = time.perf_counter() - t0
+    nbytes = int(step.context_lens[seqs].sum()) * step.num_kv_heads * step.head_dim * 4
+    return dt, nbytes
+
+
+def prepare_oracle(step):
+    import oracle
+    kc, vc = step.k_pool.copy(), step.v_pool.copy()
+    oracle.store_kvcache(kc, vc, step.k_new, step.v_new, step.slot_mapping)
+    step._ora_k, step._ora_v = kc, vc
+
+
+def cpu_baseline(step, budget_s: float = 12.0) -> dict:
+    """The oracle on as many whole sequences (in a fixed shuffled order) as fit in about
+    budget_s seconds; GB/s counts each sampled sequence's K/V bytes."""
+    prepare_oracle(step)
+    order = np.random.default_rng(0).permutation(step.batch)
+    tot_t, tot_b, n = 0.0, 0, 0
+    while n < step.batch and tot_t < budget_s:
+        dt, nb = oracle_decode_sample(step, order[n:n + 4])
+        tot_t += dt
+        tot_b += nb
+        n += len(order[n:n + 4])
+    return dict(value=tot_b / tot_t / 1e9, unit="GB/s", cores=blas_threads(), kind="oracle",
+                sample=f"{n} of {step.batch} sequences (fixed shuffled order), float64 numpy, "
+                       f"{tot_t:.1f} s; seq-steps/s {n / tot_t:.3f}")
+
+
+def run_reference(args) -> int:
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    from synth import WORKLOADS
+    step = WORKLOADS[args.workload]()
+    prepare_oracle(step)
+    order = np.random.default_rng(0).permutation(step.batch)
+    per_step = 4
+    times, nbytes = [], []
+    for i in range(args.warmup + args.steps):
+        seqs = order[(i * per_step) % step.batch:][:per_step]
+        dt, nb = oracle_decode_sample(step, seqs)
+        if i >= args.warmup:
+            times.append(dt)
+            nbytes.append(nb)
+    t = float(np.sum(times))
+    value = float(np.sum(nbytes)) / t / 1e9
+    cores = blas_threads()
+    line = dict(metric=METRIC, value=value, unit="GB/s", n_gpus=args.gpus, steps=args.steps,
+                warmup=args.warmup, ms_per_step=t / args.steps * 1e3, higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
+                impl="reference",
+                config=dict(workload=args.workload, sample_sequences_per_step=per_step),
+                cpu_baseline=dict(value=value, unit="GB/s", cores=cores, kind="oracle",
+                                  sample=f"{per_step} sequences of {step.batch} per step"),
+                e2e=dict(value=value, unit="GB/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------------
+# the GPU arm
+# ----------------------------------------------------------------------------------
+
+def run_nvpa(args) -> int:
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_422_b200 as nvpa
+    from synth import WORKLOADS
+    from synth.device import decode_to_device
+
+    world, rank, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    lib = nvpa.lib()
+
+    step = WORKLOADS[args.workload]()
+    if hasattr(step, "cu_seqlens_q"):
+        raise SystemExit("the bench step is a decode workload; prefill is measured in tests/profiles")
+    work = decode_step_bytes(step)
+    t = decode_to_device(step, dev)
+    stream = torch.cuda.Stream(device=dev)
+    ws_bytes = nvpa.paged_decode_workspace_size(step.batch, step.num_q_heads, step.num_kv_heads,
+                                                step.head_dim, step.max_context_len,
+                                                step.block_size, args.num_splits)
+    workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    out = torch.empty_like(t["q"])
+
+    def one_step(ev=None):
+        nvpa.store_kvcache(t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], t["slot_mapping"],
+                           stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        nvpa.paged_decode_attention(t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                                    t["context_lens"], step.max_context_len, step.scale, out=out,
+                                    workspace=workspace, num_splits=args.num_splits, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            one_step()
+    torch.cuda.synchronize(dev)
+
+    # ---------------- timed region: K steps, device-timed ----------------
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+        barrier(dev)
+        torch.cuda.synchronize(dev)
+        n0 = lib.nvpa_kernel_launch_count()
+        start.record(stream)
+        for i in range(args.steps):
+            one_step(evs[i])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+        launches = lib.nvpa_kernel_launch_count() - n0
+        barrier(dev)
+    ms_total = start.elapsed_time(stop)
+    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    ms_total = max_over_ranks(ms_total, dev)
+    attn_ms = max_over_ranks(attn_ms, dev)
+    ms_step = ms_total / args.steps
+
+    # ---------------- end to end: host buffers in, host result out ----------------
+    host = {k: t[k].cpu().pin_memory() for k in ("q", "k_new", "v_new", "slot_mapping",
+                                                 "block_tables", "context_lens")}
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            for k, v in host.items():
+                t[k].copy_(v, non_blocking=True)
+            one_step()
+            out_host.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+
+    peaks = measured_peaks()
+    value = work["step"] * world / (ms_step * 1e-3) / 1e9
+    attn_gbs = work["attention"] / (attn_ms * 1e-3) / 1e9
+    traffic = profile_traffic("decode_worker_b512", DECODE_SOURCES)
+    cs = clocks.summary()
+    line = dict(
+        metric=METRIC, value=value, unit="GB/s", n_gpus=world, steps=args.steps,
+        warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",
+        vs_baseline=None, dtype="bf16", data="synthetic",
+        pct_of_peak=100.0 * value / world / peaks["hbm_gbs"],
+        seq_steps_per_s=step.batch * world / (ms_step * 1e-3),
+        logical_kv_gbs=work["kv_logical"] * world / (ms_step * 1e-3) / 1e9,
+        config=dict(workload=args.workload, batch=step.batch, num_q_heads=step.num_q_heads,
+                    num_kv_heads=step.num_kv_heads, head_dim=step.head_dim,
+                    block_size=step.block_size, max_context_len=step.max_context_len,
+                    total_context_tokens=int(step.context_lens.sum()),
+                    unique_kv_bytes=work["kv_unique"], step_bytes=work["step"],
+                    parallelism=f"replicas x{world}" if world > 1 else "single GPU",
+                    l2="inputs larger than L2: %.2f GB of unique K/V per step vs 126 MB L2"
+                       % (work["kv_unique"] / 1e9),
+                    num_splits=args.num_splits),
+        roofline=dict(bound="hbm", kernel="paged_decode_attention (plan + split-KV worker + combine)",
+                      achieved=attn_gbs, peak=peaks["hbm_gbs"], unit="GB/s",
+                      frac=attn_gbs / peaks["hbm_gbs"], traffic=traffic,
+                      peak_source=peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, burst copy)"),
+        e2e=dict(value=work["step"] * world / (e2e_ms * 1e-3) / 1e9, unit="GB/s",
+                 h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=e2e_ms),
+        gpu_launches=int(launches),
+        clocks=cs,
+    )
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(step)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del t, workspace
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description="paged-KV attention benchmark (one JSON line)")
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["nvpa", "reference"], default="nvpa")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_nvpa(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

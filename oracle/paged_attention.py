@@ -57,8 +57,8 @@ PAD_SLOT = -1
 # bf16 decoding (the oracle's own; exact: every bf16 value is a float64 value)
 # ---------------------------------------------------------------------------------
 
-def bf16_to_f64(bits) -> np.ndarray:
-    """Decode uint16 bf16 bit patterns to float64 exactly.
+def _bf16_fields_to_f64(bits) -> np.ndarray:
+    """Decode uint16 bf16 bit patterns to float64 exactly, from the bit fields.
 
     A bf16 value is the upper half of an IEEE binary32 value: sign, 8 exponent bits and
     7 fraction bits.  It is decoded here from its fields, not through a float32 view.
@@ -75,6 +75,20 @@ def bf16_to_f64(bits) -> np.ndarray:
         out = np.where(special & (frac == 0), sign * np.inf, out)
         out = np.where(special & (frac != 0), np.nan, out)
     return out
+
+
+_BF16_TABLE = None
+
+
+def bf16_to_f64(bits) -> np.ndarray:
+    """Decode uint16 bf16 bit patterns to float64 exactly.
+
+    Uses a table of all 65536 patterns, each decoded once by _bf16_fields_to_f64.
+    """
+    global _BF16_TABLE
+    if _BF16_TABLE is None:
+        _BF16_TABLE = _bf16_fields_to_f64(np.arange(1 << 16, dtype=np.uint32).astype(np.uint16))
+    return _BF16_TABLE[np.asarray(bits, dtype=np.uint16)]
 
 
 # ---------------------------------------------------------------------------------

@@ -1,0 +1,68 @@
+// Host-side declarations shared by the nvpa translation units (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "nvpa.h"
+
+namespace nvpa {
+
+// printf-style message stored for nvpa_last_error() on the calling thread.
+void set_error(const char* fmt, ...);
+nvpa_status_t cuda_failure(cudaError_t e, const char* what);
+int device_sm_count();
+// Adds n to the process-wide count of kernels enqueued by the library.
+void count_launches(int n);
+
+struct DecodeCall {
+    void* out;
+    float* lse_out;
+    const void* q;
+    const void* k_cache;
+    const void* v_cache;
+    const int32_t* block_tables;
+    int max_blocks_per_seq;
+    const int32_t* context_lens;
+    int batch, hq, hkv, head_dim, num_blocks, block_size, max_context_len;
+    float scale;
+    int num_splits;
+    void* workspace;
+    size_t workspace_bytes;
+    int32_t* err_flag;
+};
+
+struct PrefillCall {
+    void* out;
+    float* lse_out;
+    const void* q;
+    const void* k_cache;
+    const void* v_cache;
+    const int32_t* block_tables;
+    int max_blocks_per_seq;
+    const int32_t* cu_seqlens_q;
+    const int32_t* cu_seqlens_k;
+    int batch, total_q, max_seqlen_q, max_seqlen_k;
+    int hq, hkv, head_dim, num_blocks, block_size;
+    float scale;
+    int causal;
+    int32_t* err_flag;
+};
+
+int decode_chunk_keys(int batch, int num_kv_heads, int max_context_len, int num_splits);
+size_t decode_workspace_bytes(int batch, int hq, int hkv, int head_dim, int max_context_len,
+                              int num_splits);
+nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream);
+nvpa_status_t run_varlen_prefill_cudacore(const PrefillCall& c, cudaStream_t stream);
+
+nvpa_status_t run_store_kvcache(const void* k, const void* v, int64_t k_stride, int64_t v_stride,
+                                void* k_cache, void* v_cache, const int32_t* slot_mapping,
+                                int num_tokens, int hkv, int head_dim, int num_blocks,
+                                int block_size, int32_t* err_flag, cudaStream_t stream);
+nvpa_status_t run_gather_kv(void* dst, const void* cache, const int32_t* block_tables,
+                            int max_blocks_per_seq, const int32_t* cu_seqlens_k, int batch,
+                            int total_k, int hkv, int head_dim, int num_blocks, int block_size,
+                            int32_t* err_flag, cudaStream_t stream);
+
+}  // namespace nvpa

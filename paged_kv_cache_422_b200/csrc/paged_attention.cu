@@ -1,0 +1,577 @@
+// Paged decode attention (split-KV + log-sum-exp combine) and the CUDA-core varlen prefill.
+//
+// Both run the same persistent, warp-specialised-by-item kernel: every warp is an
+// independent worker that takes work items (one KV head of one query row over one key
+// range), streams that range's K and V rows from the paged cache into its own ring of
+// shared-memory stages with 16-byte cp.async copies (zero-filling rows past the range,
+// never reading them), and consumes each 16-key stage with the CUDA-core tile loop of
+// attn_warp.cuh.  The issue side runs STAGES-1 tiles ahead of the consume side and
+// crosses item boundaries without draining, so a warp keeps its loads in flight from one
+// item to the next.
+//
+// Decode work items: sequence b's context is cut into partitions of `chunk` keys
+// ([P1] "Nano-vLLM part 1" 5.2: one query token per sequence reading all its cached
+// tokens).  A one-CTA plan kernel turns the device-side context lengths into a table of
+// (sequence, partition, key range) entries and resets an item counter; warps grab items
+// from the counter with atomics, so uneven context lengths balance across the SMs.
+// Items are ordered sequence-major with the KV heads of one partition adjacent, so the
+// warps reading one cache row's different heads run at the same time.  A sequence with
+// one partition is written straight to `out`; otherwise each partition writes its
+// normalised output and log-sum-exp to the workspace and a combine kernel merges them:
+//     lse = log sum_p exp(lse_p),   out = sum_p exp(lse_p - lse) * o_p.
+#include <algorithm>
+#include <mutex>
+
+#include "attn_warp.cuh"
+#include "nvpa_internal.h"
+
+namespace nvpa {
+
+constexpr int kAttnWarps = 4;
+constexpr int kAttnStages = 3;
+
+struct AttnParams {
+    const uint16_t* q;
+    const uint16_t* k_cache;
+    const uint16_t* v_cache;
+    const int32_t* block_tables;
+    const int32_t* context_lens;   // decode
+    const int32_t* cu_seqlens_q;   // prefill
+    const int32_t* cu_seqlens_k;   // prefill
+    uint16_t* out;
+    float* lse_out;
+    float* o_part;
+    float* lse_part;
+    int4* items;
+    int32_t* nsplit;
+    int32_t* counter;              // [0] next item, [1] number of items
+    int32_t* err;
+    int batch, hq, hkv, group;
+    int max_blocks, num_blocks, block_size, block_shift;
+    int max_ctx;                   // decode: max_context_len; prefill: max_seqlen_k
+    int max_q;                     // prefill: max_seqlen_q
+    int total_q;                   // prefill
+    int causal;
+    int chunk, s_max;
+    int total_static_items;        // prefill: total_q * hkv
+    float scale_log2;
+};
+
+template <int D, int GMAX>
+struct AttnStage {
+    static constexpr int KV_BYTES = kTileKeys * D * 2;
+    static constexpr int Q_BYTES = GMAX * D * 2;
+    static constexpr int BYTES = 2 * KV_BYTES + Q_BYTES + 16;
+};
+
+// ------------------------------------------------------------------------------------
+// plan: context lengths -> (sequence, partition, key range) table
+// ------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) decode_plan_kernel(const AttnParams p) {
+    __shared__ int warp_tot[32];
+    __shared__ int carry_s;
+    const int tid = threadIdx.x;
+    const int lane = tid & 31, wid = tid >> 5;
+    if (tid == 0) carry_s = 0;
+    __syncthreads();
+    const long long lim_ll = min((long long)p.max_ctx, (long long)p.max_blocks * p.block_size);
+    const int lim = (int)lim_ll;
+    for (int base = 0; base < p.batch; base += 1024) {
+        const int b = base + tid;
+        int ns = 0, ctx = 0;
+        if (b < p.batch) {
+            ctx = __ldg(p.context_lens + b);
+            if (ctx < 0 || ctx > lim) {
+                flag_error(p.err, NVPA_FLAG_BAD_LENGTH);
+                ctx = min(max(ctx, 0), lim);
+            }
+            ns = max(1, (ctx + p.chunk - 1) / p.chunk);
+            p.nsplit[b] = ns;
+        }
+        int v = ns;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int n = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += n;
+        }
+        if (lane == 31) warp_tot[wid] = v;
+        __syncthreads();
+        if (wid == 0) {
+            int w = warp_tot[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                int n = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += n;
+            }
+            warp_tot[lane] = w;
+        }
+        __syncthreads();
+        const int excl = carry_s + (v - ns) + (wid ? warp_tot[wid - 1] : 0);
+        for (int s = 0; s < ns; ++s)
+            p.items[excl + s] = make_int4(b, s | (ns << 16), s * p.chunk, min(ctx, (s + 1) * p.chunk));
+        __syncthreads();
+        if (tid == 1023) carry_s = excl + ns;
+        __syncthreads();
+    }
+    if (tid == 0) {
+        p.counter[0] = 0;
+        p.counter[1] = carry_s * p.hkv;
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// the worker kernel
+// ------------------------------------------------------------------------------------
+template <int D, int GMAX, bool PREFILL>
+__global__ void __launch_bounds__(kAttnWarps * 32)
+paged_attention_kernel(const AttnParams p) {
+    using State = WarpAttnState<D, GMAX>;
+    using Stage = AttnStage<D, GMAX>;
+    constexpr int LPR = State::LPR, RPI = State::RPI, ITER = State::ITER;
+    constexpr int STAGES = kAttnStages;
+
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int grp = lane / LPR, sub = lane % LPR;
+    uint8_t* wsm = smem + (size_t)warp * STAGES * Stage::BYTES;
+
+    const size_t row_stride = (size_t)p.hkv * D;   // elements between cache rows (slots)
+    const int bmask = p.block_size - 1;
+
+    // ---------------- issue side: the item whose tiles are being loaded ----------------
+    bool it_valid = false;
+    int it_qrow = 0, it_seq = 0, it_hk = 0, it_s = 0, it_ns = 1, it_k0 = 0, it_k1 = 0;
+    int it_ntiles = 0, it_t = 0, it_fb = 0, it_blk = -1;
+    const int32_t* it_bt = nullptr;
+
+    // decode: lane 0 holds the next item index, requested one item ahead.
+    int total_items = 0;
+    int nx_item = 0;
+    // prefill: static round-robin over items
+    int st_item = blockIdx.x * kAttnWarps + warp;
+    const int st_stride = gridDim.x * kAttnWarps;
+
+    if constexpr (!PREFILL) {
+        total_items = __ldcg(p.counter + 1);
+        if (lane == 0) nx_item = atomicAdd(p.counter, 1);
+    }
+
+    auto load_blocks = [&]() {
+        it_fb = it_k0 >> p.block_shift;
+        const int nblk = (it_k1 > it_k0) ? ((it_k1 - 1) >> p.block_shift) - it_fb + 1 : 0;
+        it_blk = -1;
+        if (lane < nblk) {
+            int e = __ldg(it_bt + it_fb + lane);
+            if (e < 0 || e >= p.num_blocks) {
+                flag_error(p.err, NVPA_FLAG_BAD_BLOCK_ID);
+                e = -1;
+            }
+            it_blk = e;
+        }
+    };
+
+    auto fetch = [&]() {
+        it_t = 0;
+        if constexpr (!PREFILL) {
+            const int idx = __shfl_sync(0xffffffffu, nx_item, 0);
+            if (idx >= total_items) {
+                it_valid = false;
+                return;
+            }
+            if (lane == 0) nx_item = atomicAdd(p.counter, 1);
+            const int4 d = __ldcg(reinterpret_cast<const int4*>(p.items) + idx / p.hkv);
+            it_valid = true;
+            it_seq = d.x;
+            it_qrow = d.x;
+            it_s = d.y & 0xffff;
+            it_ns = d.y >> 16;
+            it_k0 = d.z;
+            it_k1 = d.w;
+            it_hk = idx % p.hkv;
+        } else {
+            // prefill: item = (query token, kv head); skip tokens of malformed sequences
+            while (true) {
+                if (st_item >= p.total_static_items) {
+                    it_valid = false;
+                    return;
+                }
+                const int t = st_item / p.hkv;
+                it_hk = st_item % p.hkv;
+                st_item += st_stride;
+                // sequence of token t: last i with cu_q[i] <= t (binary search)
+                int lo = 0, hi = p.batch - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (__ldg(p.cu_seqlens_q + mid) <= t) lo = mid; else hi = mid - 1;
+                }
+                const int q0 = __ldg(p.cu_seqlens_q + lo), q1 = __ldg(p.cu_seqlens_q + lo + 1);
+                const int k0 = __ldg(p.cu_seqlens_k + lo), k1 = __ldg(p.cu_seqlens_k + lo + 1);
+                const int lq = q1 - q0, lk = k1 - k0;
+                const long long cap = (long long)p.max_blocks * p.block_size;
+                if (t < q0 || t >= q1 || lq > lk || lq > p.max_q || lk > p.max_ctx || lk > cap) {
+                    if (lane == 0 && it_hk == 0) flag_error(p.err, NVPA_FLAG_BAD_LENGTH);
+                    continue;
+                }
+                const int r = t - q0;
+                it_valid = true;
+                it_seq = lo;
+                it_qrow = t;
+                it_s = 0;
+                it_ns = 1;
+                it_k0 = 0;
+                it_k1 = p.causal ? (lk - lq + r + 1) : lk;
+                break;
+            }
+        }
+        it_bt = p.block_tables + (size_t)it_seq * p.max_blocks;
+        it_ntiles = max(1, (it_k1 - it_k0 + kTileKeys - 1) / kTileKeys);
+        load_blocks();
+    };
+
+    auto stage_ptrs = [&](int st, uint16_t*& ks, uint16_t*& vs, uint16_t*& qs, int4*& meta) {
+        uint8_t* sb = wsm + st * Stage::BYTES;
+        ks = reinterpret_cast<uint16_t*>(sb);
+        vs = ks + kTileKeys * D;
+        qs = vs + kTileKeys * D;
+        meta = reinterpret_cast<int4*>(qs + GMAX * D);
+    };
+
+    auto issue = [&](int st) {
+        uint16_t *ks, *vs, *qs;
+        int4* meta;
+        stage_ptrs(st, ks, vs, qs, meta);
+        if (!it_valid) {
+            if (lane == 0) *meta = make_int4(-1, 0, 0, 0);
+            cp_async_commit();
+            return;
+        }
+        const int key0 = it_k0 + kTileKeys * it_t;
+        int rows = min(kTileKeys, it_k1 - key0);
+        const int bi = (key0 >> p.block_shift) - it_fb;
+        int blk = __shfl_sync(0xffffffffu, it_blk, bi & 31);
+        if (bi >= 32 && rows > 0) {   // partitions longer than 32 blocks: direct lookup
+            blk = __ldg(it_bt + it_fb + bi);
+            if (blk < 0 || blk >= p.num_blocks) {
+                if (lane == 0) flag_error(p.err, NVPA_FLAG_BAD_BLOCK_ID);
+                blk = -1;
+            }
+        }
+        if (blk < 0) rows = 0;
+        rows = max(rows, 0);
+        const size_t slot0 = (size_t)max(blk, 0) * p.block_size + (key0 & bmask);
+        const uint16_t* kg = p.k_cache + slot0 * row_stride + (size_t)it_hk * D + sub * 8;
+        const uint16_t* vg = p.v_cache + slot0 * row_stride + (size_t)it_hk * D + sub * 8;
+#pragma unroll
+        for (int i = 0; i < ITER; ++i) {
+            const int r = grp + RPI * i;
+            const int nb = r < rows ? 16 : 0;
+            cp_async16(ks + r * D + sub * 8, kg + (size_t)r * row_stride, nb);
+            cp_async16(vs + r * D + sub * 8, vg + (size_t)r * row_stride, nb);
+        }
+        const bool first = it_t == 0;
+        const bool last = it_t + 1 == it_ntiles;
+        if (first) {
+            const uint16_t* qg = p.q + ((size_t)it_qrow * p.hq + (size_t)it_hk * p.group) * D;
+            for (int c = lane; c < p.group * LPR; c += 32) cp_async16(qs + c * 8, qg + c * 8, 16);
+        }
+        if (lane == 0)
+            *meta = make_int4(it_qrow, it_hk, it_s | (it_ns << 16),
+                              rows | (first ? 256 : 0) | (last ? 512 : 0));
+        cp_async_commit();
+        if (last) fetch(); else ++it_t;
+    };
+
+    State acc;
+    auto epilogue = [&](const int4 meta) {
+        acc.finish();
+        const int qrow = meta.x, hk = meta.y, s = meta.z & 0xffff, ns = meta.z >> 16;
+        if (grp != 0) return;
+#pragma unroll
+        for (int g = 0; g < GMAX; ++g) {
+            if (g >= p.group) break;
+            const int h = hk * p.group + g;
+            const float inv = acc.l[g] > 0.f ? 1.f / acc.l[g] : 0.f;
+            const float lse = acc.lse(g);
+            if (ns == 1) {
+                uint4 w;
+                w.x = pack_bf16x2(acc.o[g][0] * inv, acc.o[g][1] * inv);
+                w.y = pack_bf16x2(acc.o[g][2] * inv, acc.o[g][3] * inv);
+                w.z = pack_bf16x2(acc.o[g][4] * inv, acc.o[g][5] * inv);
+                w.w = pack_bf16x2(acc.o[g][6] * inv, acc.o[g][7] * inv);
+                *reinterpret_cast<uint4*>(p.out + ((size_t)qrow * p.hq + h) * D + sub * 8) = w;
+                if (sub == 0 && p.lse_out != nullptr) p.lse_out[(size_t)qrow * p.hq + h] = lse;
+            } else {
+                float* op = p.o_part + (((size_t)qrow * p.hq + h) * p.s_max + s) * D + sub * 8;
+                *reinterpret_cast<float4*>(op) =
+                    make_float4(acc.o[g][0] * inv, acc.o[g][1] * inv, acc.o[g][2] * inv, acc.o[g][3] * inv);
+                *reinterpret_cast<float4*>(op + 4) =
+                    make_float4(acc.o[g][4] * inv, acc.o[g][5] * inv, acc.o[g][6] * inv, acc.o[g][7] * inv);
+                if (sub == 0) p.lse_part[((size_t)qrow * p.hq + h) * p.s_max + s] = lse;
+            }
+        }
+    };
+
+    auto consume = [&](int st) -> bool {
+        uint16_t *ks, *vs, *qs;
+        int4* meta_p;
+        stage_ptrs(st, ks, vs, qs, meta_p);
+        const int4 meta = *meta_p;
+        if (meta.x < 0) return false;
+        const int rows = meta.w & 255;
+        if (meta.w & 256) {
+            acc.reset();
+            acc.load_q(qs, p.group, sub, p.scale_log2);
+        }
+        acc.consume(ks, vs, rows, lane);
+        if (meta.w & 512) epilogue(meta);
+        return true;
+    };
+
+    fetch();
+#pragma unroll
+    for (int s = 0; s < STAGES - 1; ++s) issue(s);
+    int cs = 0, is = STAGES - 1;
+    while (true) {
+        cp_async_wait<STAGES - 2>();
+        __syncwarp();
+        issue(is);
+        is = (is + 1 == STAGES) ? 0 : is + 1;
+        if (!consume(cs)) break;
+        cs = (cs + 1 == STAGES) ? 0 : cs + 1;
+    }
+    cp_async_wait<0>();
+}
+
+// ------------------------------------------------------------------------------------
+// combine: merge the partitions of every (sequence, query head) that has more than one
+// ------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) decode_combine_kernel(const AttnParams p) {
+    constexpr int DPL = D / 32;
+    const int w = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (w >= p.batch * p.hq) return;
+    const int b = w / p.hq;
+    const int ns = __ldcg(p.nsplit + b);
+    if (ns <= 1) return;
+    const float* lp = p.lse_part + (size_t)w * p.s_max;
+    float mx = -INFINITY;
+    for (int s = lane; s < ns; s += 32) mx = fmaxf(mx, __ldcg(lp + s));
+    mx = warp_max(mx);
+    float acc[DPL];
+#pragma unroll
+    for (int k = 0; k < DPL; ++k) acc[k] = 0.f;
+    float tot = 0.f;
+    if (mx > -INFINITY) {
+        for (int s0 = 0; s0 < ns; s0 += 32) {
+            const float wl = (s0 + lane < ns) ? __expf(__ldcg(lp + s0 + lane) - mx) : 0.f;
+            tot += wl;
+            const int n = min(32, ns - s0);
+            for (int j = 0; j < n; ++j) {
+                const float ws = __shfl_sync(0xffffffffu, wl, j);
+                const float* op = p.o_part + ((size_t)w * p.s_max + s0 + j) * D + lane * DPL;
+                if constexpr (DPL == 4) {
+                    const float4 o4 = __ldcg(reinterpret_cast<const float4*>(op));
+                    acc[0] = fmaf(ws, o4.x, acc[0]);
+                    acc[1] = fmaf(ws, o4.y, acc[1]);
+                    acc[2] = fmaf(ws, o4.z, acc[2]);
+                    acc[3] = fmaf(ws, o4.w, acc[3]);
+                } else {
+                    const float2 o2 = __ldcg(reinterpret_cast<const float2*>(op));
+                    acc[0] = fmaf(ws, o2.x, acc[0]);
+                    acc[1] = fmaf(ws, o2.y, acc[1]);
+                }
+            }
+        }
+        tot = warp_sum(tot);
+    }
+    const float inv = tot > 0.f ? 1.f / tot : 0.f;
+    uint16_t* dst = p.out + (size_t)w * D + lane * DPL;
+    if constexpr (DPL == 4) {
+        uint2 v;
+        v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+        v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+        *reinterpret_cast<uint2*>(dst) = v;
+    } else {
+        *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    }
+    if (lane == 0 && p.lse_out != nullptr) p.lse_out[w] = tot > 0.f ? mx + __logf(tot) : -INFINITY;
+}
+
+// ------------------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------------------
+namespace {
+
+template <int D, int GMAX, bool PREFILL>
+int worker_ctas_per_sm() {
+    static std::once_flag once[64];
+    static int cached[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    dev &= 63;
+    std::call_once(once[dev], [&] {
+        const int smem = kAttnWarps * kAttnStages * AttnStage<D, GMAX>::BYTES;
+        auto kern = paged_attention_kernel<D, GMAX, PREFILL>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kAttnWarps * 32, smem) != cudaSuccess)
+            n = 1;
+        cached[dev] = std::max(1, n);
+    });
+    return cached[dev];
+}
+
+template <int D, int GMAX, bool PREFILL>
+cudaError_t launch_worker(const AttnParams& p, long long max_items, cudaStream_t stream) {
+    const int per_sm = worker_ctas_per_sm<D, GMAX, PREFILL>();
+    const long long want = (max_items + kAttnWarps - 1) / kAttnWarps;
+    const int grid = (int)std::max(1LL, std::min<long long>((long long)device_sm_count() * per_sm, want));
+    const int smem = kAttnWarps * kAttnStages * AttnStage<D, GMAX>::BYTES;
+    paged_attention_kernel<D, GMAX, PREFILL><<<grid, kAttnWarps * 32, smem, stream>>>(p);
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) count_launches(1);
+    return e;
+}
+
+template <bool PREFILL>
+cudaError_t dispatch_worker(const AttnParams& p, int head_dim, long long max_items, cudaStream_t s) {
+    const int g = p.group;
+    const int gmax = g <= 1 ? 1 : g <= 2 ? 2 : g <= 4 ? 4 : 8;
+#define NVPA_CASE(DD, GG) \
+    if (head_dim == DD && gmax == GG) return launch_worker<DD, GG, PREFILL>(p, max_items, s);
+    NVPA_CASE(128, 1) NVPA_CASE(128, 2) NVPA_CASE(128, 4) NVPA_CASE(128, 8)
+    NVPA_CASE(64, 1) NVPA_CASE(64, 2) NVPA_CASE(64, 4) NVPA_CASE(64, 8)
+#undef NVPA_CASE
+    return cudaErrorInvalidValue;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct DecodeWorkspace {
+    size_t counter, nsplit, items, lse_part, o_part, total;
+};
+
+DecodeWorkspace decode_workspace_layout(int batch, int hq, int head_dim, int s_max) {
+    DecodeWorkspace w;
+    size_t off = 0;
+    w.counter = off; off += 256;
+    w.nsplit = off; off = align256(off + sizeof(int32_t) * (size_t)batch);
+    w.items = off; off = align256(off + sizeof(int4) * (size_t)batch * s_max);
+    w.lse_part = off;
+    off = align256(off + (s_max > 1 ? sizeof(float) * (size_t)batch * hq * s_max : 0));
+    w.o_part = off;
+    off = align256(off + (s_max > 1 ? sizeof(float) * (size_t)batch * hq * s_max * head_dim : 0));
+    w.total = off;
+    return w;
+}
+
+}  // namespace
+
+// Keys per decode partition.  Depends on host-side values only.
+int decode_chunk_keys(int batch, int num_kv_heads, int max_context_len, int num_splits) {
+    const int ctx = std::max(1, max_context_len);
+    if (num_splits > 0) {
+        const int per = (ctx + num_splits - 1) / num_splits;
+        return std::max(kTileKeys, (per + kTileKeys - 1) / kTileKeys * kTileKeys);
+    }
+    (void)batch;
+    (void)num_kv_heads;
+    return 256;
+}
+
+size_t decode_workspace_bytes(int batch, int hq, int hkv, int head_dim, int max_context_len,
+                              int num_splits) {
+    const int chunk = decode_chunk_keys(batch, hkv, max_context_len, num_splits);
+    const int s_max = std::max(1, (std::max(0, max_context_len) + chunk - 1) / chunk);
+    return decode_workspace_layout(batch, hq, head_dim, s_max).total;
+}
+
+nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream) {
+    const int chunk = decode_chunk_keys(c.batch, c.hkv, c.max_context_len, c.num_splits);
+    const int s_max = std::max(1, (std::max(0, c.max_context_len) + chunk - 1) / chunk);
+    const DecodeWorkspace w = decode_workspace_layout(c.batch, c.hq, c.head_dim, s_max);
+    if (c.workspace_bytes < w.total) {
+        set_error("workspace too small: %zu bytes given, %zu needed", c.workspace_bytes, w.total);
+        return NVPA_ERR_WORKSPACE_TOO_SMALL;
+    }
+    uint8_t* ws = static_cast<uint8_t*>(c.workspace);
+    AttnParams p{};
+    p.q = static_cast<const uint16_t*>(c.q);
+    p.k_cache = static_cast<const uint16_t*>(c.k_cache);
+    p.v_cache = static_cast<const uint16_t*>(c.v_cache);
+    p.block_tables = c.block_tables;
+    p.context_lens = c.context_lens;
+    p.out = static_cast<uint16_t*>(c.out);
+    p.lse_out = c.lse_out;
+    p.counter = reinterpret_cast<int32_t*>(ws + w.counter);
+    p.nsplit = reinterpret_cast<int32_t*>(ws + w.nsplit);
+    p.items = reinterpret_cast<int4*>(ws + w.items);
+    p.lse_part = reinterpret_cast<float*>(ws + w.lse_part);
+    p.o_part = reinterpret_cast<float*>(ws + w.o_part);
+    p.err = c.err_flag;
+    p.batch = c.batch;
+    p.hq = c.hq;
+    p.hkv = c.hkv;
+    p.group = c.hq / c.hkv;
+    p.max_blocks = c.max_blocks_per_seq;
+    p.num_blocks = c.num_blocks;
+    p.block_size = c.block_size;
+    p.block_shift = __builtin_ctz((unsigned)c.block_size);
+    p.max_ctx = c.max_context_len;
+    p.chunk = chunk;
+    p.s_max = s_max;
+    p.scale_log2 = c.scale * kLog2e;
+
+    decode_plan_kernel<<<1, 1024, 0, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_failure(e, "decode plan launch");
+    count_launches(1);
+    const long long max_items = (long long)c.batch * c.hkv * s_max;
+    e = dispatch_worker<false>(p, c.head_dim, max_items, stream);
+    if (e != cudaSuccess) return cuda_failure(e, "decode worker launch");
+    if (s_max > 1) {
+        const long long warps = (long long)c.batch * c.hq;
+        const int grid = (int)((warps + 7) / 8);
+        if (c.head_dim == 128) decode_combine_kernel<128><<<grid, 256, 0, stream>>>(p);
+        else decode_combine_kernel<64><<<grid, 256, 0, stream>>>(p);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_failure(e, "decode combine launch");
+        count_launches(1);
+    }
+    return NVPA_OK;
+}
+
+nvpa_status_t run_varlen_prefill_cudacore(const PrefillCall& c, cudaStream_t stream) {
+    AttnParams p{};
+    p.q = static_cast<const uint16_t*>(c.q);
+    p.k_cache = static_cast<const uint16_t*>(c.k_cache);
+    p.v_cache = static_cast<const uint16_t*>(c.v_cache);
+    p.block_tables = c.block_tables;
+    p.cu_seqlens_q = c.cu_seqlens_q;
+    p.cu_seqlens_k = c.cu_seqlens_k;
+    p.out = static_cast<uint16_t*>(c.out);
+    p.lse_out = c.lse_out;
+    p.err = c.err_flag;
+    p.batch = c.batch;
+    p.hq = c.hq;
+    p.hkv = c.hkv;
+    p.group = c.hq / c.hkv;
+    p.max_blocks = c.max_blocks_per_seq;
+    p.num_blocks = c.num_blocks;
+    p.block_size = c.block_size;
+    p.block_shift = __builtin_ctz((unsigned)c.block_size);
+    p.max_ctx = c.max_seqlen_k;
+    p.max_q = c.max_seqlen_q;
+    p.total_q = c.total_q;
+    p.causal = c.causal;
+    p.total_static_items = c.total_q * c.hkv;
+    p.s_max = 1;
+    p.scale_log2 = c.scale * kLog2e;
+    if (p.total_static_items == 0 || c.batch == 0) return NVPA_OK;
+    cudaError_t e = dispatch_worker<true>(p, c.head_dim, p.total_static_items, stream);
+    if (e != cudaSuccess) return cuda_failure(e, "prefill worker launch");
+    return NVPA_OK;
+}
+
+}  // namespace nvpa

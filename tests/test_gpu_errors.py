@@ -1,0 +1,77 @@
+"""Error behaviour on the GPU: host-side statuses and device-side flags (no faults)."""
+
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_422_b200 as nvpa
+from paged_kv_cache_422_b200 import NvpaError
+from synth import make_decode_step, make_prefill_step
+from synth.device import decode_to_device, i32, prefill_to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def test_unsupported_head_dim_is_rejected(cuda_device):
+    q = torch.zeros((2, 4, 96), dtype=torch.bfloat16, device=cuda_device)
+    kc = torch.zeros((4, 16, 2, 96), dtype=torch.bfloat16, device=cuda_device)
+    bt = torch.zeros((2, 1), dtype=torch.int32, device=cuda_device)
+    ctx = torch.ones(2, dtype=torch.int32, device=cuda_device)
+    with pytest.raises(NvpaError) as ei:
+        nvpa.paged_decode_attention(q, kc, kc, bt, ctx, 16, 0.1)
+    assert ei.value.status == 2
+
+
+def test_workspace_too_small_is_rejected(cuda_device):
+    step = make_decode_step(1, [4000, 10], num_q_heads=4, num_kv_heads=2, head_dim=128,
+                            block_size=256)
+    t = decode_to_device(step, cuda_device)
+    ws = torch.empty(64, dtype=torch.uint8, device=cuda_device)
+    with pytest.raises(NvpaError) as ei:
+        nvpa.paged_decode_attention(t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                                    t["context_lens"], 4000, step.scale, workspace=ws)
+    assert ei.value.status == 4
+
+
+def test_bad_block_id_is_flagged_not_read(cuda_device):
+    step = make_decode_step(2, [40, 40], num_q_heads=4, num_kv_heads=2, head_dim=64,
+                            block_size=16)
+    t = decode_to_device(step, cuda_device)
+    nvpa.store_kvcache(t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], t["slot_mapping"])
+    t["block_tables"][1, 1] = step.num_blocks + 5
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    out = nvpa.paged_decode_attention(t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                                      t["context_lens"], 40, step.scale, err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() & nvpa.NVPA_FLAG_BAD_BLOCK_ID
+    assert torch.isfinite(out.float()).all()
+
+
+def test_context_longer_than_declared_is_flagged(cuda_device):
+    step = make_decode_step(3, [100, 20], num_q_heads=4, num_kv_heads=2, head_dim=64,
+                            block_size=16)
+    t = decode_to_device(step, cuda_device)
+    nvpa.store_kvcache(t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], t["slot_mapping"])
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    out = nvpa.paged_decode_attention(t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                                      t["context_lens"], 50, step.scale, err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() & nvpa.NVPA_FLAG_BAD_LENGTH
+    assert torch.isfinite(out.float()).all()
+
+
+def test_prefill_more_queries_than_keys_is_flagged(cuda_device):
+    step = make_prefill_step(4, [50, 30], num_q_heads=4, num_kv_heads=2, head_dim=64,
+                             block_size=16)
+    t = prefill_to_device(step, cuda_device)
+    nvpa.store_kvcache(t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], t["slot_mapping"])
+    bad_cu_k = i32([0, 40, 70], cuda_device)       # sequence 0 now has Lq 50 > Lk 40
+    out = torch.full_like(t["q"], 7.0)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    nvpa.varlen_prefill_attention(t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                                  t["cu_seqlens_q"], bad_cu_k, 50, 50, step.scale, out=out,
+                                  err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() & nvpa.NVPA_FLAG_BAD_LENGTH
+    assert torch.all(out[:50] == 7.0)                 # rows of the bad sequence untouched
+    assert torch.isfinite(out[50:].float()).all() and not torch.all(out[50:] == 7.0)

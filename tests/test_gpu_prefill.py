@@ -1,0 +1,83 @@
+"""Varlen (prefix-cached) causal prefill attention on the GPU against the float64 oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_422_b200 as nvpa
+from synth import make_decode_step, make_prefill_step, prefill_varlen_prefix_hits
+from synth.device import bf16_tensor, decode_to_device, i32, prefill_to_device
+from tests.helpers import assert_attention_close, assert_lse_close, oracle_after_store
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(step, t, causal=True, err=None):
+    nvpa.store_kvcache(t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], t["slot_mapping"],
+                       err_flag=err)
+    out, lse = nvpa.varlen_prefill_attention(
+        t["q"], t["k_cache"], t["v_cache"], t["block_tables"], t["cu_seqlens_q"],
+        t["cu_seqlens_k"], step.max_seqlen_q, step.max_seqlen_k, step.scale, causal=causal,
+        err_flag=err, return_lse=True)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+def _oracle(step, causal=True):
+    kc, vc, bad = oracle_after_store(step)
+    assert bad == []
+    return oracle.varlen_prefill_attention(step.q, kc, vc, step.block_tables, step.cu_seqlens_q,
+                                           step.cu_seqlens_k, step.scale, causal=causal)
+
+
+def test_prefill_prefix_hits_full_size(cuda_device):
+    step = prefill_varlen_prefix_hits()
+    assert (step.cached_blocks > 0).sum() > 0
+    t = prefill_to_device(step, cuda_device)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    out, lse = _run(step, t, err=err)
+    assert err.item() == 0
+    ora_out, ora_lse = _oracle(step)
+    assert_attention_close(out, ora_out, "prefill_varlen_prefix_hits_b32")
+    assert_lse_close(lse, ora_lse, "prefill_varlen_prefix_hits_b32")
+
+
+CASES = [
+    # (total lengths, cached blocks, Hq, Hkv, D, block size)
+    ([1, 2, 17, 64], [0, 0, 0, 0], 4, 2, 64, 16),
+    ([300, 129, 40], [2, 1, 0], 8, 8, 128, 64),
+    ([513, 256, 1000], [1, 1, 3], 16, 8, 128, 256),
+    ([64, 64], [4, 0], 6, 2, 128, 16),          # first sequence fully cached: Lq = 0
+    ([200, 31, 77], [3, 0, 2], 12, 4, 64, 32),
+    ([700], [1], 8, 1, 128, 128),
+]
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("lens,cached,hq,hkv,d,bs", CASES)
+def test_prefill_small_shapes(cuda_device, lens, cached, hq, hkv, d, bs, causal):
+    step = make_prefill_step(sum(lens) + bs, lens, cached_blocks=cached, num_q_heads=hq,
+                             num_kv_heads=hkv, head_dim=d, block_size=bs)
+    t = prefill_to_device(step, cuda_device)
+    out, lse = _run(step, t, causal=causal)
+    ora_out, ora_lse = _oracle(step, causal=causal)
+    assert_attention_close(out, ora_out, f"prefill {lens} causal={causal}")
+    assert_lse_close(lse, ora_lse, f"prefill {lens} causal={causal}")
+
+
+def test_prefill_last_row_equals_decode(cuda_device):
+    """The last query row of a causal prefill sees the whole context: decode of the same
+    token over the same cache gives the same attention."""
+    step = make_prefill_step(40, [333, 90], cached_blocks=[2, 1], num_q_heads=8, num_kv_heads=2,
+                             head_dim=128, block_size=32)
+    t = prefill_to_device(step, cuda_device)
+    out_p, _ = _run(step, t)
+    last = torch.as_tensor(step.cu_seqlens_q[1:] - 1, device=cuda_device, dtype=torch.long)
+    q_last = t["q"][last].contiguous()
+    out_d = nvpa.paged_decode_attention(q_last, t["k_cache"], t["v_cache"], t["block_tables"],
+                                        i32(step.seq_lens, cuda_device), int(step.seq_lens.max()),
+                                        step.scale)
+    torch.cuda.synchronize()
+    diff = (out_p[last].float() - out_d.float()).abs().max().item()
+    assert diff <= 2e-2
