@@ -238,12 +238,14 @@ def oracle_decode_sample(step, seqs):
     oracle.paged_decode_attention(step.q[seqs], step._ora_k, step._ora_v, step.block_tables[seqs],
                                   step.context_lens[seqs], step.scale)
     dt = time.perf_counter() - t0
-    nbytes = int(step.context_lens[seqs].sum()) * step.num_kv_heads * step.head_dim * 4
-    return dt, nbytes
+    # the sample's share of the step's algorithmic bytes, in proportion to context length
+    share = float(step.context_lens[seqs].sum()) / float(step.context_lens.sum())
+    return dt, step._bytes["step"] * share
 
 
 def prepare_oracle(step):
     import oracle
+    step.__dict__.setdefault("_bytes", decode_step_bytes(step))
     kc, vc = step.k_pool.copy(), step.v_pool.copy()
     oracle.store_kvcache(kc, vc, step.k_new, step.v_new, step.slot_mapping)
     step._ora_k, step._ora_v = kc, vc

@@ -79,6 +79,9 @@ typedef enum nvpa_status {
                                      [0, num_blocks): its rows are treated as absent        */
 #define NVPA_FLAG_BAD_LENGTH   4  /* a context length / cumulative length outside the bounds
                                      declared by the call: clamped to those bounds          */
+#define NVPA_FLAG_TIMEOUT      8  /* a tensor-core kernel's internal wait exceeded its time
+                                     limit (2 s): the kernel stopped early, outputs are
+                                     incomplete; never expected in correct operation        */
 
 /* Library version, as 10000*major + 100*minor + patch. */
 int nvpa_version(void);

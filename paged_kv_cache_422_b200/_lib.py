@@ -20,6 +20,7 @@ NVPA_ERR_WORKSPACE_TOO_SMALL = 4
 NVPA_FLAG_BAD_SLOT = 1
 NVPA_FLAG_BAD_BLOCK_ID = 2
 NVPA_FLAG_BAD_LENGTH = 4
+NVPA_FLAG_TIMEOUT = 8
 
 # Every function the header declares, with (restype, argtypes).
 _p = ctypes.c_void_p

@@ -48,16 +48,25 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False) -> str:
-    """Compile and link libnvpa.so; return its path."""
+def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False,
+          defines=(), out: str | None = None) -> str:
+    """Compile and link libnvpa.so; return its path.
+
+    `defines` (NAME=VALUE strings) and `out` build a variant library elsewhere, with its
+    objects in a build folder of its own (used for tuning experiments).
+    """
     nvcc = _nvcc()
-    os.makedirs(BUILD, exist_ok=True)
+    lib_path = os.path.abspath(out) if out else LIB
+    build_dir = BUILD if not defines else os.path.join(
+        BUILD, "variant_" + "_".join(d.replace("=", "-") for d in defines))
+    os.makedirs(build_dir, exist_ok=True)
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     headers = _headers()
     extra = ["-Xptxas", "-v"] if ptxas_verbose else []
+    extra += [f"-D{d}" for d in defines]
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         if force or ptxas_verbose or _stale(obj, [src] + headers):
             cmd = [nvcc, "-c", src, "-o", obj] + CFLAGS + extra
             if verbose:
@@ -71,16 +80,16 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
 
     with ThreadPoolExecutor(max_workers=min(len(sources), os.cpu_count() or 1)) as ex:
         objs = list(ex.map(compile_one, sources))
-    if force or _stale(LIB, objs):
-        tmp = LIB + ".tmp"
+    if force or _stale(lib_path, objs):
+        tmp = lib_path + ".tmp"
         cmd = [nvcc, "--shared", "-o", tmp] + objs + ARCH + ["-Xcompiler", "-fPIC"]
         if verbose:
             print(" ".join(cmd), flush=True)
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib_path)
+    return lib_path
 
 
 def main(argv=None):
@@ -89,8 +98,12 @@ def main(argv=None):
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-verbose", action="store_true",
                     help="print registers / spills / shared memory per kernel")
+    ap.add_argument("-D", "--define", action="append", default=[],
+                    help="NAME=VALUE preprocessor define for a variant build")
+    ap.add_argument("--out", default=None, help="output path of a variant library")
     a = ap.parse_args(argv)
-    print(build(force=a.force, verbose=a.verbose, ptxas_verbose=a.ptxas_verbose))
+    print(build(force=a.force, verbose=a.verbose, ptxas_verbose=a.ptxas_verbose,
+                defines=tuple(a.define), out=a.out))
 
 
 if __name__ == "__main__":

@@ -23,6 +23,32 @@
 namespace nvpa {
 
 constexpr int kTileKeys = 16;
+constexpr float kRescaleSlack = 8.0f;   // log2 units
+
+// Packed pairs of float32 in one 64-bit register pair; sm_100 executes the .f32x2 forms
+// of fma/mul as single instructions, halving the FMA count of the inner loops.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// A packed bf16 pair (low half = element 2j, high half = element 2j+1) widened exactly.
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
+    return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
 
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;
@@ -48,10 +74,10 @@ struct WarpAttnState {
     static constexpr int ITER = kTileKeys / RPI;
     static_assert(ITER * 2 == LPR, "tile shape assumes 16 keys = RPI * LPR / 2");
 
-    float q[GMAX][8];   // this lane's 8 dims of each query head, scaled to log2 units
-    float o[GMAX][8];   // running un-normalised output for the same dims
-    float m[GMAX];      // running max (log2 units), warp-uniform
-    float l[GMAX];      // running sum of weights, this lane's share
+    uint64_t q[GMAX][4];  // this lane's 8 dims of each query head as 4 packed pairs, in log2 units
+    uint64_t o[GMAX][4];  // running un-normalised output for the same dims, packed pairs
+    float m[GMAX];        // running max (log2 units), warp-uniform
+    float l[GMAX];        // running sum of weights, this lane's share
 
     __device__ __forceinline__ void reset() {
 #pragma unroll
@@ -59,7 +85,7 @@ struct WarpAttnState {
             m[g] = -INFINITY;
             l[g] = 0.f;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) o[g][k] = 0.f;
+            for (int k = 0; k < 4; ++k) o[g][k] = 0ull;
         }
     }
 
@@ -76,8 +102,13 @@ struct WarpAttnState {
                 for (int k = 0; k < 8; ++k) f[k] = 0.f;
             }
 #pragma unroll
-            for (int k = 0; k < 8; ++k) q[g][k] = f[k] * scale_log2;
+            for (int k = 0; k < 4; ++k) q[g][k] = f2_pack(f[2 * k] * scale_log2, f[2 * k + 1] * scale_log2);
         }
+    }
+
+    // Output dims 8*sub + 2k, 8*sub + 2k + 1 of head g.
+    __device__ __forceinline__ void out_pair(int g, int k, float& lo, float& hi) const {
+        f2_unpack(o[g][k], lo, hi);
     }
 
     // One halving round of the transpose-reduction: N live values, partner at lane ^ OFF.
@@ -107,15 +138,18 @@ struct WarpAttnState {
 #pragma unroll
         for (int i = 0; i < ITER; ++i) {
             const int row = grp + RPI * i;
-            uint4 u = *reinterpret_cast<const uint4*>(ks + row * D + sub * 8);
-            float f[8];
-            unpack8(u, f);
+            const uint4 u = *reinterpret_cast<const uint4*>(ks + row * D + sub * 8);
+            const uint64_t kp[4] = {bf16x2_to_f2(u.x), bf16x2_to_f2(u.y), bf16x2_to_f2(u.z),
+                                    bf16x2_to_f2(u.w)};
 #pragma unroll
             for (int g = 0; g < GMAX; ++g) {
-                float acc = q[g][0] * f[0];
-#pragma unroll
-                for (int k = 1; k < 8; ++k) acc = fmaf(q[g][k], f[k], acc);
-                part[g][i] = acc;
+                uint64_t acc = f2_mul(q[g][0], kp[0]);
+                acc = f2_fma(q[g][1], kp[1], acc);
+                acc = f2_fma(q[g][2], kp[2], acc);
+                acc = f2_fma(q[g][3], kp[3], acc);
+                float lo, hi;
+                f2_unpack(acc, lo, hi);
+                part[g][i] = lo + hi;
             }
         }
         // transpose-reduce: LPR/2 .. 2 halve the live values, the final round (offset 1)
@@ -128,41 +162,53 @@ struct WarpAttnState {
 
         const int my_row = grp + RPI * (sub >> 1);
         const bool row_ok = my_row < rows_valid;
+        // Lazy rescaling: weights are exp2(s - m) against a reference max m that moves only
+        // when some score exceeds it by more than kRescaleSlack (then o and l are rescaled).
+        // Weights stay below 2^kRescaleSlack, far from fp32 overflow, and the final o / l
+        // does not depend on which reference was used.  One warp vote replaces the per-tile
+        // max reduction in the common case.
+        float sc[GMAX];
+        bool over = false;
+#pragma unroll
+        for (int g = 0; g < GMAX; ++g) {
+            sc[g] = row_ok ? part[g][0] : -INFINITY;
+            over |= sc[g] > m[g] + kRescaleSlack;
+        }
+        if (__any_sync(0xffffffffu, over)) {
+#pragma unroll
+            for (int g = 0; g < GMAX; ++g) {
+                const float m_new = fmaxf(m[g], warp_max(sc[g]));
+                if (m_new > m[g]) {
+                    const float alpha = fast_exp2(m[g] - m_new);   // 0 when m was -inf
+                    l[g] *= alpha;
+                    const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) o[g][k] = f2_mul(o[g][k], a2);
+                    m[g] = m_new;
+                }
+            }
+        }
         float p[GMAX];
 #pragma unroll
         for (int g = 0; g < GMAX; ++g) {
-            const float s = row_ok ? part[g][0] : -INFINITY;
-            const float m_new = fmaxf(m[g], warp_max(s));
-            float alpha, pg;
-            if (m_new == -INFINITY) {
-                alpha = 1.f;
-                pg = 0.f;
-            } else {
-                alpha = fast_exp2(m[g] - m_new);
-                pg = row_ok ? fast_exp2(s - m_new) : 0.f;
-            }
+            // rows past the range and heads that saw no key yet contribute exactly zero
+            const float pg = (row_ok && m[g] > -INFINITY) ? fast_exp2(sc[g] - m[g]) : 0.f;
             p[g] = pg;
-            l[g] = l[g] * alpha + ((sub & 1) ? 0.f : pg);
-            m[g] = m_new;
-            if (alpha != 1.f) {
-#pragma unroll
-                for (int k = 0; k < 8; ++k) o[g][k] *= alpha;
-            }
+            l[g] += (sub & 1) ? 0.f : pg;
         }
 #pragma unroll
         for (int i = 0; i < ITER; ++i) {
             const int row = grp + RPI * i;
             const int owner = grp * LPR + 2 * i;
-            float w[GMAX];
-#pragma unroll
-            for (int g = 0; g < GMAX; ++g) w[g] = __shfl_sync(0xffffffffu, p[g], owner);
-            uint4 u = *reinterpret_cast<const uint4*>(vs + row * D + sub * 8);
-            float f[8];
-            unpack8(u, f);
+            const uint4 u = *reinterpret_cast<const uint4*>(vs + row * D + sub * 8);
+            const uint64_t vp[4] = {bf16x2_to_f2(u.x), bf16x2_to_f2(u.y), bf16x2_to_f2(u.z),
+                                    bf16x2_to_f2(u.w)};
 #pragma unroll
             for (int g = 0; g < GMAX; ++g) {
+                const float w = __shfl_sync(0xffffffffu, p[g], owner);
+                const uint64_t w2 = f2_pack(w, w);
 #pragma unroll
-                for (int k = 0; k < 8; ++k) o[g][k] = fmaf(w[g], f[k], o[g][k]);
+                for (int k = 0; k < 4; ++k) o[g][k] = f2_fma(w2, vp[k], o[g][k]);
             }
         }
     }
@@ -176,7 +222,13 @@ struct WarpAttnState {
 #pragma unroll
             for (int g = 0; g < GMAX; ++g) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) o[g][k] += __shfl_xor_sync(0xffffffffu, o[g][k], off);
+                for (int k = 0; k < 4; ++k) {
+                    float lo, hi;
+                    f2_unpack(o[g][k], lo, hi);
+                    lo += __shfl_xor_sync(0xffffffffu, lo, off);
+                    hi += __shfl_xor_sync(0xffffffffu, hi, off);
+                    o[g][k] = f2_pack(lo, hi);
+                }
             }
         }
 #pragma unroll

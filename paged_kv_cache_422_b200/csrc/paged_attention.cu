@@ -17,7 +17,8 @@
 // Items are ordered sequence-major with the KV heads of one partition adjacent, so the
 // warps reading one cache row's different heads run at the same time.  A sequence with
 // one partition is written straight to `out`; otherwise each partition writes its
-// normalised output and log-sum-exp to the workspace and a combine kernel merges them:
+// normalised output and log-sum-exp to the workspace and a combine kernel (one warp per
+// sequence and query head) merges them with the log-sum-exp weights:
 //     lse = log sum_p exp(lse_p),   out = sum_p exp(lse_p - lse) * o_p.
 #include <algorithm>
 #include <mutex>
@@ -27,8 +28,12 @@
 
 namespace nvpa {
 
+#ifndef NVPA_DECODE_STAGES
+#define NVPA_DECODE_STAGES 2
+#endif
+
 constexpr int kAttnWarps = 4;
-constexpr int kAttnStages = 3;
+constexpr int kAttnStages = NVPA_DECODE_STAGES;
 
 struct AttnParams {
     const uint16_t* q;
@@ -285,28 +290,30 @@ paged_attention_kernel(const AttnParams p) {
     auto epilogue = [&](const int4 meta) {
         acc.finish();
         const int qrow = meta.x, hk = meta.y, s = meta.z & 0xffff, ns = meta.z >> 16;
-        if (grp != 0) return;
+        if (grp == 0) {
 #pragma unroll
-        for (int g = 0; g < GMAX; ++g) {
-            if (g >= p.group) break;
-            const int h = hk * p.group + g;
-            const float inv = acc.l[g] > 0.f ? 1.f / acc.l[g] : 0.f;
-            const float lse = acc.lse(g);
-            if (ns == 1) {
-                uint4 w;
-                w.x = pack_bf16x2(acc.o[g][0] * inv, acc.o[g][1] * inv);
-                w.y = pack_bf16x2(acc.o[g][2] * inv, acc.o[g][3] * inv);
-                w.z = pack_bf16x2(acc.o[g][4] * inv, acc.o[g][5] * inv);
-                w.w = pack_bf16x2(acc.o[g][6] * inv, acc.o[g][7] * inv);
-                *reinterpret_cast<uint4*>(p.out + ((size_t)qrow * p.hq + h) * D + sub * 8) = w;
-                if (sub == 0 && p.lse_out != nullptr) p.lse_out[(size_t)qrow * p.hq + h] = lse;
-            } else {
-                float* op = p.o_part + (((size_t)qrow * p.hq + h) * p.s_max + s) * D + sub * 8;
-                *reinterpret_cast<float4*>(op) =
-                    make_float4(acc.o[g][0] * inv, acc.o[g][1] * inv, acc.o[g][2] * inv, acc.o[g][3] * inv);
-                *reinterpret_cast<float4*>(op + 4) =
-                    make_float4(acc.o[g][4] * inv, acc.o[g][5] * inv, acc.o[g][6] * inv, acc.o[g][7] * inv);
-                if (sub == 0) p.lse_part[((size_t)qrow * p.hq + h) * p.s_max + s] = lse;
+            for (int g = 0; g < GMAX; ++g) {
+                if (g >= p.group) break;
+                const int h = hk * p.group + g;
+                const float inv = acc.l[g] > 0.f ? 1.f / acc.l[g] : 0.f;
+                const float lse = acc.lse(g);
+                float v[8];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) acc.out_pair(g, k, v[2 * k], v[2 * k + 1]);
+                if (ns == 1) {
+                    uint4 w;
+                    w.x = pack_bf16x2(v[0] * inv, v[1] * inv);
+                    w.y = pack_bf16x2(v[2] * inv, v[3] * inv);
+                    w.z = pack_bf16x2(v[4] * inv, v[5] * inv);
+                    w.w = pack_bf16x2(v[6] * inv, v[7] * inv);
+                    *reinterpret_cast<uint4*>(p.out + ((size_t)qrow * p.hq + h) * D + sub * 8) = w;
+                    if (sub == 0 && p.lse_out != nullptr) p.lse_out[(size_t)qrow * p.hq + h] = lse;
+                } else {
+                    float* op = p.o_part + (((size_t)qrow * p.hq + h) * p.s_max + s) * D + sub * 8;
+                    __stcg(reinterpret_cast<float4*>(op), make_float4(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv));
+                    __stcg(reinterpret_cast<float4*>(op + 4), make_float4(v[4] * inv, v[5] * inv, v[6] * inv, v[7] * inv));
+                    if (sub == 0) __stcg(p.lse_part + ((size_t)qrow * p.hq + h) * p.s_max + s, lse);
+                }
             }
         }
     };
@@ -347,7 +354,7 @@ paged_attention_kernel(const AttnParams p) {
 // ------------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) decode_combine_kernel(const AttnParams p) {
-    constexpr int DPL = D / 32;
+    constexpr int DPL = D / 32;   // output dims per lane
     const int w = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (w >= p.batch * p.hq) return;
@@ -355,6 +362,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const AttnParams p)
     const int ns = __ldcg(p.nsplit + b);
     if (ns <= 1) return;
     const float* lp = p.lse_part + (size_t)w * p.s_max;
+    const float* op = p.o_part + (size_t)w * p.s_max * D + lane * DPL;
     float mx = -INFINITY;
     for (int s = lane; s < ns; s += 32) mx = fmaxf(mx, __ldcg(lp + s));
     mx = warp_max(mx);
@@ -364,23 +372,35 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const AttnParams p)
     float tot = 0.f;
     if (mx > -INFINITY) {
         for (int s0 = 0; s0 < ns; s0 += 32) {
-            const float wl = (s0 + lane < ns) ? __expf(__ldcg(lp + s0 + lane) - mx) : 0.f;
+            const float wl = (s0 + lane < ns) ? fast_exp2((__ldcg(lp + s0 + lane) - mx) * kLog2e) : 0.f;
             tot += wl;
             const int n = min(32, ns - s0);
-            for (int j = 0; j < n; ++j) {
-                const float ws = __shfl_sync(0xffffffffu, wl, j);
-                const float* op = p.o_part + ((size_t)w * p.s_max + s0 + j) * D + lane * DPL;
-                if constexpr (DPL == 4) {
-                    const float4 o4 = __ldcg(reinterpret_cast<const float4*>(op));
-                    acc[0] = fmaf(ws, o4.x, acc[0]);
-                    acc[1] = fmaf(ws, o4.y, acc[1]);
-                    acc[2] = fmaf(ws, o4.z, acc[2]);
-                    acc[3] = fmaf(ws, o4.w, acc[3]);
-                } else {
-                    const float2 o2 = __ldcg(reinterpret_cast<const float2*>(op));
-                    acc[0] = fmaf(ws, o2.x, acc[0]);
-                    acc[1] = fmaf(ws, o2.y, acc[1]);
+            int j = 0;
+            for (; j + 4 <= n; j += 4) {   // four independent loads in flight
+                float ws[4];
+                float v[4][DPL];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    ws[u] = __shfl_sync(0xffffffffu, wl, j + u);
+                    const float* src = op + (size_t)(s0 + j + u) * D;
+                    if constexpr (DPL == 4) {
+                        const float4 t = __ldcg(reinterpret_cast<const float4*>(src));
+                        v[u][0] = t.x; v[u][1] = t.y; v[u][2] = t.z; v[u][3] = t.w;
+                    } else {
+                        const float2 t = __ldcg(reinterpret_cast<const float2*>(src));
+                        v[u][0] = t.x; v[u][1] = t.y;
+                    }
                 }
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int k = 0; k < DPL; ++k) acc[k] = fmaf(ws[u], v[u][k], acc[k]);
+            }
+            for (; j < n; ++j) {
+                const float ws = __shfl_sync(0xffffffffu, wl, j);
+                const float* src = op + (size_t)(s0 + j) * D;
+#pragma unroll
+                for (int k = 0; k < DPL; ++k) acc[k] = fmaf(ws, __ldcg(src + k), acc[k]);
             }
         }
         tot = warp_sum(tot);
@@ -452,7 +472,8 @@ struct DecodeWorkspace {
     size_t counter, nsplit, items, lse_part, o_part, total;
 };
 
-DecodeWorkspace decode_workspace_layout(int batch, int hq, int head_dim, int s_max) {
+DecodeWorkspace decode_workspace_layout(int batch, int hq, int hkv, int head_dim, int s_max) {
+    (void)hkv;
     DecodeWorkspace w;
     size_t off = 0;
     w.counter = off; off += 256;
@@ -484,13 +505,13 @@ size_t decode_workspace_bytes(int batch, int hq, int hkv, int head_dim, int max_
                               int num_splits) {
     const int chunk = decode_chunk_keys(batch, hkv, max_context_len, num_splits);
     const int s_max = std::max(1, (std::max(0, max_context_len) + chunk - 1) / chunk);
-    return decode_workspace_layout(batch, hq, head_dim, s_max).total;
+    return decode_workspace_layout(batch, hq, hkv, head_dim, s_max).total;
 }
 
 nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream) {
     const int chunk = decode_chunk_keys(c.batch, c.hkv, c.max_context_len, c.num_splits);
     const int s_max = std::max(1, (std::max(0, c.max_context_len) + chunk - 1) / chunk);
-    const DecodeWorkspace w = decode_workspace_layout(c.batch, c.hq, c.head_dim, s_max);
+    const DecodeWorkspace w = decode_workspace_layout(c.batch, c.hq, c.hkv, c.head_dim, s_max);
     if (c.workspace_bytes < w.total) {
         set_error("workspace too small: %zu bytes given, %zu needed", c.workspace_bytes, w.total);
         return NVPA_ERR_WORKSPACE_TOO_SMALL;
