@@ -175,6 +175,37 @@ nvpa_status_t nvpa_paged_decode_attention(void* out, float* lse_out, const void*
                                           int32_t* err_flag, cudaStream_t stream);
 
 /*
+ * nvpa_paged_decode_attention_static_scratch -- the same decode attention for callers
+ * that cannot allocate device memory: a plugin inside a host runtime whose memory
+ * manager owns all device memory and offers no allocation hook, or code running where an
+ * allocation is not allowed (a cudaMalloc there fails, or synchronises the device and
+ * stalls queued work).  No page describes this: it is an interface addition with no
+ * counterpart in the method.
+ *
+ * Arguments and results are those of nvpa_paged_decode_attention without
+ * workspace/workspace_bytes.  The scratch the decode needs (partition plan and split
+ * partials) lives in a fixed 64 MiB array compiled into the library; every GPU that
+ * loads the library holds those 64 MiB until the process exits.  The call allocates
+ * nothing (no cudaMalloc, no cudaFree, no allocating library routine).
+ *  - The first call on a device resolves the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call before any
+ *    stream capture.
+ *  - A call whose scratch need (nvpa_paged_decode_workspace_size with the same
+ *    arguments) exceeds 64 MiB returns NVPA_ERR_WORKSPACE_TOO_SMALL with a message;
+ *    lowering num_splits lowers the need (batch 512 at max_context_len 4096 with 16 query
+ *    heads of dim 128 fits with num_splits <= 15).
+ *  - All calls share the one array, which keeps the last call's contents.  Nothing in it
+ *    has to start at zero.  Calls whose kernels can overlap on the GPU (different streams
+ *    or threads) race on the array: serialise them.
+ */
+nvpa_status_t nvpa_paged_decode_attention_static_scratch(
+    void* out, float* lse_out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+    int batch, int num_q_heads, int num_kv_heads, int head_dim, int num_blocks,
+    int block_size, int max_context_len, float softmax_scale, int num_splits,
+    int32_t* err_flag, cudaStream_t stream);
+
+/*
  * nvpa_varlen_prefill_attention -- [P1] 5.2 prefill preparation (cumulative sequence
  * lengths) and [P3] "Low-level performance details" (varlen attention in prefill),
  * with prefix caching ([P1] 4.2): sequence i owns query rows
