@@ -322,7 +322,7 @@ def run_nvpa(args) -> int:
 
     step = WORKLOADS[args.workload]()
     if hasattr(step, "cu_seqlens_q"):
-        raise SystemExit("the bench step is a decode workload; prefill is measured in tests/profiles")
+        return run_nvpa_prefill(args, step, dev, lib, world, rank)
     work = decode_step_bytes(step)
     t = decode_to_device(step, dev)
     stream = torch.cuda.Stream(device=dev)
@@ -430,6 +430,82 @@ def run_nvpa(args) -> int:
     if rank == 0:
         print(json.dumps(line), flush=True)
     del t, workspace
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
+    """A prefill step: store the uncached suffix tokens, then varlen causal attention.
+    value = algorithmic causal FLOPs / step time (TFLOP/s)."""
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_422_b200 as nvpa
+    from synth.device import prefill_to_device
+
+    work = prefill_step_work(step)
+    t = prefill_to_device(step, dev)
+    stream = torch.cuda.Stream(device=dev)
+    ws = torch.empty(nvpa.varlen_prefill_workspace_size(step.batch, step.total_q),
+                     dtype=torch.uint8, device=dev)
+    out = torch.empty_like(t["q"])
+
+    def one_step(ev=None):
+        nvpa.store_kvcache(t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], t["slot_mapping"],
+                           stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        nvpa.varlen_prefill_attention(t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                                      t["cu_seqlens_q"], t["cu_seqlens_k"], step.max_seqlen_q,
+                                      step.max_seqlen_k, step.scale, out=out, workspace=ws,
+                                      stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            one_step()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+        barrier(dev)
+        torch.cuda.synchronize(dev)
+        n0 = lib.nvpa_kernel_launch_count()
+        start.record(stream)
+        for i in range(args.steps):
+            one_step(evs[i])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+        launches = lib.nvpa_kernel_launch_count() - n0
+        barrier(dev)
+    ms_step = max_over_ranks(start.elapsed_time(stop) / args.steps, dev)
+    attn_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in evs])), dev)
+    peaks = measured_peaks()
+    tflops = work["flops"] * world / (ms_step * 1e-3) / 1e12
+    attn_tflops = work["flops"] / (attn_ms * 1e-3) / 1e12
+    line = dict(
+        metric="varlen causal prefill with prefix-cache hits: TFLOP/s (algorithmic causal FLOPs)",
+        value=tflops, unit="TFLOP/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
+        ms_per_step=ms_step, higher_is_better=True, scaling="weak", vs_baseline=None,
+        dtype="bf16", data="synthetic",
+        tokens_per_s=step.total_q * world / (ms_step * 1e-3),
+        store_gbs=work["store"] / ((ms_step - attn_ms) * 1e-3) / 1e9 if ms_step > attn_ms else None,
+        config=dict(workload=args.workload, batch=step.batch, total_q=step.total_q,
+                    max_seqlen_q=step.max_seqlen_q, max_seqlen_k=step.max_seqlen_k,
+                    num_q_heads=step.num_q_heads, num_kv_heads=step.num_kv_heads,
+                    head_dim=step.head_dim, block_size=step.block_size,
+                    algorithmic_tflop=work["flops"] / 1e12,
+                    l2="not flushed: K/V of the step (about 140 MB) is near the 126 MB L2"),
+        roofline=dict(bound="tensor", kernel="varlen_prefill_attention (plan + tcgen05 kernel)",
+                      achieved=attn_tflops, peak=peaks["bf16_tflops"], unit="TFLOP/s",
+                      frac=attn_tflops / peaks["bf16_tflops"], traffic=None,
+                      peak_source=peaks["source"] + " (MEASURED_PEAKS.json bf16_tflops, burst)"),
+        gpu_launches=int(launches), clocks=clocks.summary())
+    if rank == 0:
+        print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
     return 0

@@ -206,6 +206,12 @@ nvpa_status_t nvpa_paged_decode_attention_static_scratch(
     int32_t* err_flag, cudaStream_t stream);
 
 /*
+ * Workspace for nvpa_varlen_prefill_attention, in bytes (the query-tile schedule), for a
+ * call with `batch` sequences and `total_q` query rows.  Host-side values only.
+ */
+size_t nvpa_varlen_prefill_workspace_size(int batch, int total_q);
+
+/*
  * nvpa_varlen_prefill_attention -- [P1] 5.2 prefill preparation (cumulative sequence
  * lengths) and [P3] "Low-level performance details" (varlen attention in prefill),
  * with prefix caching ([P1] 4.2): sequence i owns query rows
@@ -224,6 +230,13 @@ nvpa_status_t nvpa_paged_decode_attention_static_scratch(
  *                   Lk <= max_blocks_per_seq*block_size, cu_seqlens_q[batch] = total_q.
  *                   A violation is flagged (NVPA_FLAG_BAD_LENGTH) and that sequence's
  *                   rows are left unwritten.
+ *   workspace       device scratch of at least nvpa_varlen_prefill_workspace_size(batch,
+ *                   total_q) bytes, 256-byte aligned, no initialisation needed; calls that
+ *                   share a workspace must not overlap.
+ * A block-table entry outside [0, num_blocks) is flagged (NVPA_FLAG_BAD_BLOCK_ID), its
+ * rows are not loaded, and that sequence's output is unspecified (finite).
+ * QK^T and PV run on the tensor cores (tcgen05, bf16 inputs, fp32 accumulation in TMEM);
+ * P is rounded to bf16 before the PV product.
  * Errors: as for decode.
  */
 nvpa_status_t nvpa_varlen_prefill_attention(void* out, float* lse_out, const void* q,
@@ -236,6 +249,7 @@ nvpa_status_t nvpa_varlen_prefill_attention(void* out, float* lse_out, const voi
                                             int num_q_heads, int num_kv_heads, int head_dim,
                                             int num_blocks, int block_size,
                                             float softmax_scale, int causal,
+                                            void* workspace, size_t workspace_bytes,
                                             int32_t* err_flag, cudaStream_t stream);
 
 /*

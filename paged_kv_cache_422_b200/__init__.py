@@ -10,6 +10,7 @@ from ._lib import (  # noqa: F401
     NVPA_FLAG_BAD_BLOCK_ID,
     NVPA_FLAG_BAD_LENGTH,
     NVPA_FLAG_BAD_SLOT,
+    NVPA_FLAG_TIMEOUT,
     NvpaError,
     lib,
 )
@@ -19,4 +20,5 @@ from .api import (  # noqa: F401
     paged_decode_workspace_size,
     store_kvcache,
     varlen_prefill_attention,
+    varlen_prefill_workspace_size,
 )

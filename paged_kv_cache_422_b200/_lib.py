@@ -39,8 +39,9 @@ SIGNATURES = {
                                          _i, _f, _i, _p, _sz, _p, _p]),
     "nvpa_paged_decode_attention_static_scratch": (_i, [_p, _p, _p, _p, _p, _p, _i, _p, _i, _i,
                                                         _i, _i, _i, _i, _i, _f, _i, _p, _p]),
+    "nvpa_varlen_prefill_workspace_size": (_sz, [_i, _i]),
     "nvpa_varlen_prefill_attention": (_i, [_p, _p, _p, _p, _p, _p, _i, _p, _p, _i, _i, _i, _i,
-                                           _i, _i, _i, _i, _i, _f, _i, _p, _p]),
+                                           _i, _i, _i, _i, _i, _f, _i, _p, _sz, _p, _p]),
     "nvpa_gather_kv": (_i, [_p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _p, _p]),
 }
 

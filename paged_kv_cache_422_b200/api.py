@@ -114,9 +114,14 @@ def paged_decode_attention(q, k_cache, v_cache, block_tables, context_lens, max_
     return (out, lse) if return_lse else out
 
 
+def varlen_prefill_workspace_size(batch, total_q) -> int:
+    return int(lib().nvpa_varlen_prefill_workspace_size(batch, total_q))
+
+
 def varlen_prefill_attention(q, k_cache, v_cache, block_tables, cu_seqlens_q, cu_seqlens_k,
                              max_seqlen_q, max_seqlen_k, softmax_scale, causal=True, out=None,
-                             lse=None, err_flag=None, stream=None, return_lse=False):
+                             lse=None, workspace=None, err_flag=None, stream=None,
+                             return_lse=False):
     """Varlen (prefix-cached) causal prefill: q [total_q, Hq, D] bf16; keys of sequence i
     are 0..Lk-1 read through block_tables[i]."""
     nb, bs, hkv, d = _cache_dims(k_cache, v_cache)
@@ -134,11 +139,15 @@ def varlen_prefill_attention(q, k_cache, v_cache, block_tables, cu_seqlens_q, cu
         out = torch.empty_like(q)
     if return_lse and lse is None:
         lse = torch.empty((total_q, hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(varlen_prefill_workspace_size(batch, total_q), dtype=torch.uint8,
+                                device=q.device)
     st = lib().nvpa_varlen_prefill_attention(
         _ptr(out), _ptr(lse), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
         int(block_tables.shape[1]), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), batch, total_q,
         int(max_seqlen_q), int(max_seqlen_k), hq, hkv, d, nb, bs, float(softmax_scale),
-        1 if causal else 0, _ptr(err_flag), _stream_handle(stream))
+        1 if causal else 0, _ptr(workspace), int(workspace.numel() * workspace.element_size()),
+        _ptr(err_flag), _stream_handle(stream))
     check(st, "nvpa_varlen_prefill_attention")
     return (out, lse) if return_lse else out
 

@@ -165,6 +165,11 @@ nvpa_status_t nvpa_paged_decode_attention(void* out, float* lse_out, const void*
     return run_paged_decode(c, stream);
 }
 
+size_t nvpa_varlen_prefill_workspace_size(int batch, int total_q) {
+    if (batch < 0 || total_q < 0) return 0;
+    return prefill_workspace_bytes(batch, total_q);
+}
+
 nvpa_status_t nvpa_varlen_prefill_attention(void* out, float* lse_out, const void* q,
                                             const void* k_cache, const void* v_cache,
                                             const int32_t* block_tables, int max_blocks_per_seq,
@@ -172,7 +177,8 @@ nvpa_status_t nvpa_varlen_prefill_attention(void* out, float* lse_out, const voi
                                             int batch, int total_q, int max_seqlen_q,
                                             int max_seqlen_k, int num_q_heads, int num_kv_heads,
                                             int head_dim, int num_blocks, int block_size,
-                                            float softmax_scale, int causal, int32_t* err_flag,
+                                            float softmax_scale, int causal, void* workspace,
+                                            size_t workspace_bytes, int32_t* err_flag,
                                             cudaStream_t stream) {
     g_last_error[0] = 0;
     NVPA_REQUIRE(batch >= 0 && total_q >= 0 && max_seqlen_q >= 0 && max_seqlen_k >= 0,
@@ -185,14 +191,17 @@ nvpa_status_t nvpa_varlen_prefill_attention(void* out, float* lse_out, const voi
     NVPA_REQUIRE((long long)total_q * num_kv_heads <= 0x7fffffffLL, NVPA_ERR_UNSUPPORTED,
                  "total_q * num_kv_heads above 2^31-1");
     if (batch == 0 || total_q == 0) return NVPA_OK;
-    NVPA_REQUIRE(out && q && k_cache && v_cache && block_tables && cu_seqlens_q && cu_seqlens_k,
+    NVPA_REQUIRE(out && q && k_cache && v_cache && block_tables && cu_seqlens_q && cu_seqlens_k &&
+                     workspace,
                  NVPA_ERR_INVALID_ARG, "null pointer");
     NVPA_REQUIRE(aligned16(out) && aligned16(q) && aligned16(k_cache) && aligned16(v_cache),
                  NVPA_ERR_INVALID_ARG, "bf16 pointers must be 16-byte aligned");
+    NVPA_REQUIRE((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0, NVPA_ERR_INVALID_ARG,
+                 "workspace must be 256-byte aligned");
     PrefillCall c{out, lse_out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, cu_seqlens_q,
                   cu_seqlens_k, batch, total_q, max_seqlen_q, max_seqlen_k, num_q_heads, num_kv_heads,
                   head_dim, num_blocks, block_size, softmax_scale, causal, err_flag};
-    return run_varlen_prefill_cudacore(c, stream);
+    return run_varlen_prefill_tcgen05(c, workspace, workspace_bytes, stream);
 }
 
 nvpa_status_t nvpa_gather_kv(void* dst, const void* cache, const int32_t* block_tables,

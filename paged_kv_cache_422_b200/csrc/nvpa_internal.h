@@ -54,7 +54,9 @@ int decode_chunk_keys(int batch, int num_kv_heads, int max_context_len, int num_
 size_t decode_workspace_bytes(int batch, int hq, int hkv, int head_dim, int max_context_len,
                               int num_splits);
 nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream);
-nvpa_status_t run_varlen_prefill_cudacore(const PrefillCall& c, cudaStream_t stream);
+size_t prefill_workspace_bytes(int batch, int total_q);
+nvpa_status_t run_varlen_prefill_tcgen05(const PrefillCall& c, void* workspace, size_t workspace_bytes,
+                                         cudaStream_t stream);
 
 nvpa_status_t run_store_kvcache(const void* k, const void* v, int64_t k_stride, int64_t v_stride,
                                 void* k_cache, void* v_cache, const int32_t* slot_mapping,

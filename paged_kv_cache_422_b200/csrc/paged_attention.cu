@@ -1,24 +1,23 @@
-// Paged decode attention (split-KV + log-sum-exp combine) and the CUDA-core varlen prefill.
+// Paged decode attention: split-KV partitions merged by log-sum-exp.
 //
-// Both run the same persistent, warp-specialised-by-item kernel: every warp is an
-// independent worker that takes work items (one KV head of one query row over one key
-// range), streams that range's K and V rows from the paged cache into its own ring of
-// shared-memory stages with 16-byte cp.async copies (zero-filling rows past the range,
-// never reading them), and consumes each 16-key stage with the CUDA-core tile loop of
-// attn_warp.cuh.  The issue side runs STAGES-1 tiles ahead of the consume side and
-// crosses item boundaries without draining, so a warp keeps its loads in flight from one
-// item to the next.
+// The worker kernel is persistent and every warp is an independent worker: it takes
+// work items (one KV head of one partition of one sequence's context), streams that
+// range's K and V rows from the paged cache into its own ring of shared-memory stages
+// with 16-byte cp.async copies (zero-filling rows past the range, never reading them),
+// and consumes each 16-key stage with the CUDA-core tile loop of attn_warp.cuh.  The
+// issue side runs STAGES-1 tiles ahead of the consume side and crosses item boundaries
+// without draining, so a warp keeps its loads in flight from one item to the next.
 //
-// Decode work items: sequence b's context is cut into partitions of `chunk` keys
-// ([P1] "Nano-vLLM part 1" 5.2: one query token per sequence reading all its cached
-// tokens).  A one-CTA plan kernel turns the device-side context lengths into a table of
-// (sequence, partition, key range) entries and resets an item counter; warps grab items
-// from the counter with atomics, so uneven context lengths balance across the SMs.
-// Items are ordered sequence-major with the KV heads of one partition adjacent, so the
-// warps reading one cache row's different heads run at the same time.  A sequence with
-// one partition is written straight to `out`; otherwise each partition writes its
-// normalised output and log-sum-exp to the workspace and a combine kernel (one warp per
-// sequence and query head) merges them with the log-sum-exp weights:
+// Work items: sequence b's context is cut into partitions of `chunk` keys ("Nano-vLLM
+// part 1" section 5.2: one query token per sequence reading all its cached tokens).  A
+// one-CTA plan kernel turns the device-side context lengths into a table of (sequence,
+// partition, key range) entries and resets an item counter; warps grab items from the
+// counter with atomics, so uneven context lengths balance across the SMs.  Items are
+// ordered sequence-major with the KV heads of one partition adjacent, so the warps
+// reading one cache row's different heads run at the same time.  A sequence with one
+// partition is written straight to `out`; otherwise each partition writes its normalised
+// output and log-sum-exp to the workspace and a combine kernel (one warp per sequence
+// and query head) merges them with the log-sum-exp weights:
 //     lse = log sum_p exp(lse_p),   out = sum_p exp(lse_p - lse) * o_p.
 #include <algorithm>
 #include <mutex>
@@ -40,9 +39,7 @@ struct AttnParams {
     const uint16_t* k_cache;
     const uint16_t* v_cache;
     const int32_t* block_tables;
-    const int32_t* context_lens;   // decode
-    const int32_t* cu_seqlens_q;   // prefill
-    const int32_t* cu_seqlens_k;   // prefill
+    const int32_t* context_lens;
     uint16_t* out;
     float* lse_out;
     float* o_part;
@@ -53,12 +50,8 @@ struct AttnParams {
     int32_t* err;
     int batch, hq, hkv, group;
     int max_blocks, num_blocks, block_size, block_shift;
-    int max_ctx;                   // decode: max_context_len; prefill: max_seqlen_k
-    int max_q;                     // prefill: max_seqlen_q
-    int total_q;                   // prefill
-    int causal;
-    int chunk, s_max;
-    int total_static_items;        // prefill: total_q * hkv
+    int max_ctx;                   // host-side bound of context_lens
+    int chunk, s_max;              // keys per partition, partitions of the longest context
     float scale_log2;
 };
 
@@ -127,7 +120,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const AttnParams p) {
 // ------------------------------------------------------------------------------------
 // the worker kernel
 // ------------------------------------------------------------------------------------
-template <int D, int GMAX, bool PREFILL>
+template <int D, int GMAX>
 __global__ void __launch_bounds__(kAttnWarps * 32)
 paged_attention_kernel(const AttnParams p) {
     using State = WarpAttnState<D, GMAX>;
@@ -149,17 +142,10 @@ paged_attention_kernel(const AttnParams p) {
     int it_ntiles = 0, it_t = 0, it_fb = 0, it_blk = -1;
     const int32_t* it_bt = nullptr;
 
-    // decode: lane 0 holds the next item index, requested one item ahead.
-    int total_items = 0;
+    // Lane 0 holds the next item index, requested one item ahead.
+    const int total_items = __ldcg(p.counter + 1);
     int nx_item = 0;
-    // prefill: static round-robin over items
-    int st_item = blockIdx.x * kAttnWarps + warp;
-    const int st_stride = gridDim.x * kAttnWarps;
-
-    if constexpr (!PREFILL) {
-        total_items = __ldcg(p.counter + 1);
-        if (lane == 0) nx_item = atomicAdd(p.counter, 1);
-    }
+    if (lane == 0) nx_item = atomicAdd(p.counter, 1);
 
     auto load_blocks = [&]() {
         it_fb = it_k0 >> p.block_shift;
@@ -177,57 +163,21 @@ paged_attention_kernel(const AttnParams p) {
 
     auto fetch = [&]() {
         it_t = 0;
-        if constexpr (!PREFILL) {
-            const int idx = __shfl_sync(0xffffffffu, nx_item, 0);
-            if (idx >= total_items) {
-                it_valid = false;
-                return;
-            }
-            if (lane == 0) nx_item = atomicAdd(p.counter, 1);
-            const int4 d = __ldcg(reinterpret_cast<const int4*>(p.items) + idx / p.hkv);
-            it_valid = true;
-            it_seq = d.x;
-            it_qrow = d.x;
-            it_s = d.y & 0xffff;
-            it_ns = d.y >> 16;
-            it_k0 = d.z;
-            it_k1 = d.w;
-            it_hk = idx % p.hkv;
-        } else {
-            // prefill: item = (query token, kv head); skip tokens of malformed sequences
-            while (true) {
-                if (st_item >= p.total_static_items) {
-                    it_valid = false;
-                    return;
-                }
-                const int t = st_item / p.hkv;
-                it_hk = st_item % p.hkv;
-                st_item += st_stride;
-                // sequence of token t: last i with cu_q[i] <= t (binary search)
-                int lo = 0, hi = p.batch - 1;
-                while (lo < hi) {
-                    const int mid = (lo + hi + 1) >> 1;
-                    if (__ldg(p.cu_seqlens_q + mid) <= t) lo = mid; else hi = mid - 1;
-                }
-                const int q0 = __ldg(p.cu_seqlens_q + lo), q1 = __ldg(p.cu_seqlens_q + lo + 1);
-                const int k0 = __ldg(p.cu_seqlens_k + lo), k1 = __ldg(p.cu_seqlens_k + lo + 1);
-                const int lq = q1 - q0, lk = k1 - k0;
-                const long long cap = (long long)p.max_blocks * p.block_size;
-                if (t < q0 || t >= q1 || lq > lk || lq > p.max_q || lk > p.max_ctx || lk > cap) {
-                    if (lane == 0 && it_hk == 0) flag_error(p.err, NVPA_FLAG_BAD_LENGTH);
-                    continue;
-                }
-                const int r = t - q0;
-                it_valid = true;
-                it_seq = lo;
-                it_qrow = t;
-                it_s = 0;
-                it_ns = 1;
-                it_k0 = 0;
-                it_k1 = p.causal ? (lk - lq + r + 1) : lk;
-                break;
-            }
+        const int idx = __shfl_sync(0xffffffffu, nx_item, 0);
+        if (idx >= total_items) {
+            it_valid = false;
+            return;
         }
+        if (lane == 0) nx_item = atomicAdd(p.counter, 1);
+        const int4 d = __ldcg(reinterpret_cast<const int4*>(p.items) + idx / p.hkv);
+        it_valid = true;
+        it_seq = d.x;
+        it_qrow = d.x;
+        it_s = d.y & 0xffff;
+        it_ns = d.y >> 16;
+        it_k0 = d.z;
+        it_k1 = d.w;
+        it_hk = idx % p.hkv;
         it_bt = p.block_tables + (size_t)it_seq * p.max_blocks;
         it_ntiles = max(1, (it_k1 - it_k0 + kTileKeys - 1) / kTileKeys);
         load_blocks();
@@ -423,7 +373,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const AttnParams p)
 // ------------------------------------------------------------------------------------
 namespace {
 
-template <int D, int GMAX, bool PREFILL>
+template <int D, int GMAX>
 int worker_ctas_per_sm() {
     static std::once_flag once[64];
     static int cached[64];
@@ -432,7 +382,7 @@ int worker_ctas_per_sm() {
     dev &= 63;
     std::call_once(once[dev], [&] {
         const int smem = kAttnWarps * kAttnStages * AttnStage<D, GMAX>::BYTES;
-        auto kern = paged_attention_kernel<D, GMAX, PREFILL>;
+        auto kern = paged_attention_kernel<D, GMAX>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         int n = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kAttnWarps * 32, smem) != cudaSuccess)
@@ -442,24 +392,23 @@ int worker_ctas_per_sm() {
     return cached[dev];
 }
 
-template <int D, int GMAX, bool PREFILL>
+template <int D, int GMAX>
 cudaError_t launch_worker(const AttnParams& p, long long max_items, cudaStream_t stream) {
-    const int per_sm = worker_ctas_per_sm<D, GMAX, PREFILL>();
+    const int per_sm = worker_ctas_per_sm<D, GMAX>();
     const long long want = (max_items + kAttnWarps - 1) / kAttnWarps;
     const int grid = (int)std::max(1LL, std::min<long long>((long long)device_sm_count() * per_sm, want));
     const int smem = kAttnWarps * kAttnStages * AttnStage<D, GMAX>::BYTES;
-    paged_attention_kernel<D, GMAX, PREFILL><<<grid, kAttnWarps * 32, smem, stream>>>(p);
+    paged_attention_kernel<D, GMAX><<<grid, kAttnWarps * 32, smem, stream>>>(p);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
     return e;
 }
 
-template <bool PREFILL>
 cudaError_t dispatch_worker(const AttnParams& p, int head_dim, long long max_items, cudaStream_t s) {
     const int g = p.group;
     const int gmax = g <= 1 ? 1 : g <= 2 ? 2 : g <= 4 ? 4 : 8;
 #define NVPA_CASE(DD, GG) \
-    if (head_dim == DD && gmax == GG) return launch_worker<DD, GG, PREFILL>(p, max_items, s);
+    if (head_dim == DD && gmax == GG) return launch_worker<DD, GG>(p, max_items, s);
     NVPA_CASE(128, 1) NVPA_CASE(128, 2) NVPA_CASE(128, 4) NVPA_CASE(128, 8)
     NVPA_CASE(64, 1) NVPA_CASE(64, 2) NVPA_CASE(64, 4) NVPA_CASE(64, 8)
 #undef NVPA_CASE
@@ -549,7 +498,7 @@ nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream) {
     if (e != cudaSuccess) return cuda_failure(e, "decode plan launch");
     count_launches(1);
     const long long max_items = (long long)c.batch * c.hkv * s_max;
-    e = dispatch_worker<false>(p, c.head_dim, max_items, stream);
+    e = dispatch_worker(p, c.head_dim, max_items, stream);
     if (e != cudaSuccess) return cuda_failure(e, "decode worker launch");
     if (s_max > 1) {
         const long long warps = (long long)c.batch * c.hq;
@@ -560,38 +509,6 @@ nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream) {
         if (e != cudaSuccess) return cuda_failure(e, "decode combine launch");
         count_launches(1);
     }
-    return NVPA_OK;
-}
-
-nvpa_status_t run_varlen_prefill_cudacore(const PrefillCall& c, cudaStream_t stream) {
-    AttnParams p{};
-    p.q = static_cast<const uint16_t*>(c.q);
-    p.k_cache = static_cast<const uint16_t*>(c.k_cache);
-    p.v_cache = static_cast<const uint16_t*>(c.v_cache);
-    p.block_tables = c.block_tables;
-    p.cu_seqlens_q = c.cu_seqlens_q;
-    p.cu_seqlens_k = c.cu_seqlens_k;
-    p.out = static_cast<uint16_t*>(c.out);
-    p.lse_out = c.lse_out;
-    p.err = c.err_flag;
-    p.batch = c.batch;
-    p.hq = c.hq;
-    p.hkv = c.hkv;
-    p.group = c.hq / c.hkv;
-    p.max_blocks = c.max_blocks_per_seq;
-    p.num_blocks = c.num_blocks;
-    p.block_size = c.block_size;
-    p.block_shift = __builtin_ctz((unsigned)c.block_size);
-    p.max_ctx = c.max_seqlen_k;
-    p.max_q = c.max_seqlen_q;
-    p.total_q = c.total_q;
-    p.causal = c.causal;
-    p.total_static_items = c.total_q * c.hkv;
-    p.s_max = 1;
-    p.scale_log2 = c.scale * kLog2e;
-    if (p.total_static_items == 0 || c.batch == 0) return NVPA_OK;
-    cudaError_t e = dispatch_worker<true>(p, c.head_dim, p.total_static_items, stream);
-    if (e != cudaSuccess) return cuda_failure(e, "prefill worker launch");
     return NVPA_OK;
 }
 

@@ -1,0 +1,648 @@
+// Varlen causal prefill attention on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+// ("Nano-vLLM inference engine architecture", section "Low-level performance details":
+// prefill runs a variable-length attention over cumulative sequence lengths; "Nano-vLLM
+// part 1" section 5.2 builds those lengths; section 4.2's prefix caching means the keys
+// of a sequence are its cached prefix followed by the suffix stored in this step.)
+//
+// Work unit: a tile of 128 query rows against one KV head.  The rows are 128/P tokens of
+// one sequence times the P query heads (P = query heads per KV head when that is a power
+// of two up to 8, else 1) that share the KV head, so each K/V tile fetched serves P
+// heads.  Keys come in tiles of 128 from the block-paged cache.  With a causal mask the
+// unit only visits key tiles up to its last token's position (bottom-right alignment:
+// suffix token r is at position Lk - Lq + r).
+//
+// A one-CTA plan kernel lists the (sequence, query tile) pairs, longest first (by key
+// tiles visited).  The attention kernel is persistent with two CTAs per SM, so that one
+// CTA's softmax overlaps the other's MMAs; CTA c takes list entries c, c + gridDim.x, ...
+// for every KV head.  Inside a CTA the warps have roles:
+//   warp 0      TMA producer: the Q tile, then K_j and V_j tiles into a 2-stage ring
+//               (one 3-D tensor-map box per cache block piece; a 128-key tile spans
+//               128 / block_size blocks when the block size is below 128);
+//   warp 1      allocates 256 TMEM columns; one lane issues the MMAs:
+//                 S_j = Q K_j^T   (SS: both operands in shared memory, K-major)
+//                 O  += P_j V_j   (TS: P from TMEM, V from shared memory, MN-major);
+//   warps 2..5  softmax, one thread per query row: read S_j from TMEM 32 columns at a
+//               time, mask, exponentiate against the current reference max, keep P_j
+//               packed in registers; only when some score exceeds the reference by more
+//               than 2^8 (always on the first tile) the reference moves, O is rescaled
+//               in TMEM and P_j is recomputed from S_j; then P_j is written as bf16 over
+//               S_j.  At the end O is divided by the row sum and stored with the lse.
+// TMEM columns: S/P [0, 128), O [128, 128 + D).  The MMAs of one thread execute in issue
+// order, so S_{j+1} (issued after O += P_j V_j) cannot overwrite P_j early.
+//
+// Stale rows (freed blocks are not cleared, part 1 section 4.3): K rows past the length
+// are masked in the softmax by select (never by arithmetic), and V rows past the length
+// in the last key tile are zeroed in shared memory before their MMA, so a 0 weight never
+// meets a NaN.
+#include <algorithm>
+#include <mutex>
+
+#include "attn_warp.cuh"
+#include "nvpa_internal.h"
+#include "sm100.cuh"
+
+namespace nvpa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kQ = 128;          // query rows per tile (MMA M): tokens x packed heads
+constexpr int kKV = 128;         // keys per tile (MMA N of QK^T, K of PV)
+constexpr int kStages = 2;       // K/V ring stages, each one K or one V tile
+constexpr int kThreads = 192;    // 6 warps
+constexpr int kTmemCols = 256;   // S/P 128 + O up to 128
+constexpr int kMinTokensPerTile = 16;   // 128 rows / at most 8 packed heads
+
+struct PrefillParams {
+    const int32_t* block_tables;
+    const int32_t* cu_q;
+    const int32_t* cu_k;
+    uint16_t* out;
+    float* lse_out;
+    int32_t* err;
+    const int2* tiles;           // plan: (sequence, query tile), longest first
+    const int32_t* ntiles;       // plan: number of entries
+    int batch, total_q, hq, hkv, group;
+    int pack, pack_shift;        // query heads per row group (P) and log2(P)
+    int tq;                      // tokens per tile, 128 / P
+    int hgroups;                 // head groups, hq / P
+    int max_blocks, num_blocks, block_size, block_shift;
+    int max_q, max_k, causal;
+    float scale_log2;
+};
+
+template <int D>
+struct Layout {
+    static constexpr int REGIONS = D / 64;                  // 64 bf16 = one 128-byte swizzle row
+    static constexpr int REGION_BYTES = 128 * 128;          // 128 rows x 128 bytes
+    static constexpr int TILE_BYTES = REGIONS * REGION_BYTES;
+    static constexpr int Q_OFF = 0;
+    static constexpr int STAGE_OFF = TILE_BYTES;
+    static constexpr int BAR_OFF = STAGE_OFF + kStages * TILE_BYTES;
+    // barriers
+    static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_KVFULL = 2, B_KVEMPTY = B_KVFULL + kStages;
+    static constexpr int B_SFULL = B_KVEMPTY + kStages, B_PFULL = B_SFULL + 1;
+    static constexpr int B_ODONE = B_PFULL + 1, B_OFINAL = B_ODONE + 1, B_OFREE = B_OFINAL + 1;
+    static constexpr int B_DRAIN = B_OFREE + 1, NBARS = B_DRAIN + 1;
+    static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;     // tmem base, abort flag
+    static constexpr int BYTES = MISC_OFF + 16;
+    static constexpr int ALLOC = BYTES + 1024;               // room to align the base to 1024
+};
+
+struct TileInfo {
+    int seq, qt, head0, hk;
+    int q0, lq, lk;      // first query row (global), query rows, keys of the sequence
+    int tok0, ntok;      // first token of the tile inside the sequence, tokens in the tile
+    int nkv;             // key tiles visited
+};
+
+__device__ __forceinline__ int tile_nkv(int causal, int lq, int lk, int tok0, int ntok) {
+    const int ktiles = (lk + kKV - 1) / kKV;
+    return causal ? min(ktiles, (lk - lq + tok0 + ntok - 1) / kKV + 1) : ktiles;
+}
+
+__device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, int idx) {
+    TileInfo t;
+    const int2 e = __ldg(p.tiles + idx / p.hgroups);
+    t.seq = e.x;
+    t.qt = e.y;
+    t.head0 = (idx % p.hgroups) * p.pack;
+    t.hk = t.head0 / p.group;
+    t.q0 = __ldg(p.cu_q + t.seq);
+    t.lq = __ldg(p.cu_q + t.seq + 1) - t.q0;
+    t.lk = __ldg(p.cu_k + t.seq + 1) - __ldg(p.cu_k + t.seq);
+    t.tok0 = t.qt * p.tq;
+    t.ntok = min(p.tq, t.lq - t.tok0);
+    t.nkv = tile_nkv(p.causal, t.lq, t.lk, t.tok0, t.ntok);
+    return t;
+}
+
+// ------------------------------------------------------------------------------------
+// plan: list (sequence, query tile) pairs, most key tiles first
+// ------------------------------------------------------------------------------------
+constexpr int kPlanBins = 1024;
+
+__global__ void __launch_bounds__(1024) prefill_plan_kernel(const PrefillParams p, int2* tiles,
+                                                            int32_t* ntiles) {
+    __shared__ int hist[kPlanBins];
+    __shared__ int cursor[kPlanBins];
+    const int tid = threadIdx.x;
+    for (int i = tid; i < kPlanBins; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const long long cap = (long long)p.max_blocks * p.block_size;
+    auto seq_ok = [&](int i, int& lq, int& lk) {
+        const int q0 = __ldg(p.cu_q + i), q1 = __ldg(p.cu_q + i + 1);
+        const int k0 = __ldg(p.cu_k + i), k1 = __ldg(p.cu_k + i + 1);
+        lq = q1 - q0;
+        lk = k1 - k0;
+        return q0 >= 0 && lq >= 0 && lk >= lq && lq <= p.max_q && lk <= p.max_k && lk <= cap &&
+               q1 <= p.total_q;
+    };
+    auto nkv_of = [&](int lq, int lk, int qt) {
+        const int tok0 = qt * p.tq;
+        return min(max(tile_nkv(p.causal, lq, lk, tok0, min(p.tq, lq - tok0)), 0), kPlanBins - 1);
+    };
+    for (int i = tid; i < p.batch; i += blockDim.x) {
+        int lq, lk;
+        if (!seq_ok(i, lq, lk)) {
+            flag_error(p.err, NVPA_FLAG_BAD_LENGTH);
+            continue;
+        }
+        for (int qt = 0; qt * p.tq < lq; ++qt) atomicAdd(&hist[nkv_of(lq, lk, qt)], 1);
+    }
+    __syncthreads();
+    if (tid == 0) {   // descending prefix: most key tiles first
+        int acc = 0;
+        for (int b = kPlanBins - 1; b >= 0; --b) {
+            cursor[b] = acc;
+            acc += hist[b];
+        }
+        *ntiles = acc;
+    }
+    __syncthreads();
+    for (int i = tid; i < p.batch; i += blockDim.x) {
+        int lq, lk;
+        if (!seq_ok(i, lq, lk)) continue;
+        for (int qt = 0; qt * p.tq < lq; ++qt) {
+            const int pos = atomicAdd(&cursor[nkv_of(lq, lk, qt)], 1);
+            tiles[pos] = make_int2(i, qt);
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// the attention kernel
+// ------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kThreads, 2)
+prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap k_map,
+                       const __grid_constant__ CUtensorMap v_map, const PrefillParams p) {
+    using L = Layout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
+    const uint32_t sbase = smem_u32(smem);
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bars + L::B_QFULL, 1);
+        mbar_init(bars + L::B_QEMPTY, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bars + L::B_KVFULL + s, 1);
+            mbar_init(bars + L::B_KVEMPTY + s, 1);
+        }
+        mbar_init(bars + L::B_SFULL, 1);
+        mbar_init(bars + L::B_PFULL, 4);
+        mbar_init(bars + L::B_ODONE, 1);
+        mbar_init(bars + L::B_OFINAL, 1);
+        mbar_init(bars + L::B_OFREE, 4);
+        mbar_init(bars + L::B_DRAIN, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&q_map);
+        tma_prefetch_desc(&k_map);
+        tma_prefetch_desc(&v_map);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t TM_S = 0, TM_O = kKV;   // column offsets
+
+    const int total = __ldcg(p.ntiles) * p.hgroups;
+
+    if (warp == 0) {
+        // ============================ TMA producer ============================
+        if (lane == 0) {
+            uint32_t fill = 0;
+            int tcount = 0;
+            int last_fill[kStages];
+            for (int s = 0; s < kStages; ++s) last_fill[s] = -1;
+            for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
+                const TileInfo t = tile_info(p, idx);
+                if (!mbar_wait(bars + L::B_QEMPTY, (tcount & 1) ^ 1, abort_flag, p.err)) break;
+                mbar_arrive_expect_tx(bars + L::B_QFULL, L::TILE_BYTES);
+                for (int r = 0; r < L::REGIONS; ++r)
+                    tma_load_3d(smem + L::Q_OFF + r * L::REGION_BYTES, &q_map, bars + L::B_QFULL, r * 64,
+                                t.head0, t.q0 + t.tok0);
+                const int32_t* bt = p.block_tables + (size_t)t.seq * p.max_blocks;
+                const int piece = min(p.block_size, kKV);
+                bool ok = true;
+                for (int j = 0; j < t.nkv && ok; ++j) {
+                    const int key0 = j * kKV;
+                    const int nrows = min(kKV, t.lk - key0);
+                    const int npieces = (nrows + piece - 1) / piece;
+                    for (int kv = 0; kv < 2; ++kv) {
+                        const int slot = fill % kStages;
+                        if (!mbar_wait(bars + L::B_KVEMPTY + slot, ((fill / kStages) & 1) ^ 1, abort_flag, p.err)) {
+                            ok = false;
+                            break;
+                        }
+                        uint8_t* dst = smem + L::STAGE_OFF + slot * L::TILE_BYTES;
+                        uint32_t bytes = 0;
+                        int blks[kKV / 16];
+                        for (int c = 0; c < npieces; ++c) {
+                            const int kc = key0 + c * piece;
+                            int blk = __ldg(bt + (kc >> p.block_shift));
+                            if (blk < 0 || blk >= p.num_blocks) {
+                                flag_error(p.err, NVPA_FLAG_BAD_BLOCK_ID);
+                                blk = -1;
+                            } else {
+                                bytes += (uint32_t)(piece * 128 * L::REGIONS);
+                            }
+                            blks[c] = blk;
+                        }
+                        mbar_arrive_expect_tx(bars + L::B_KVFULL + slot, bytes);
+                        const CUtensorMap* map = kv ? &v_map : &k_map;
+                        for (int c = 0; c < npieces; ++c) {
+                            if (blks[c] < 0) continue;
+                            const int kc = key0 + c * piece;
+                            const int z = blks[c] * p.block_size + (kc & (p.block_size - 1));
+                            for (int r = 0; r < L::REGIONS; ++r)
+                                tma_load_3d(dst + r * L::REGION_BYTES + c * piece * 128, map,
+                                            bars + L::B_KVFULL + slot, r * 64, t.hk, z);
+                        }
+                        last_fill[slot] = (int)fill;
+                        ++fill;
+                    }
+                }
+                ++tcount;
+                if (!ok) break;
+            }
+            // let every copy this thread started land before the CTA can exit
+            for (int s = 0; s < kStages; ++s) {
+                if (last_fill[s] < 0) continue;
+                const uint64_t t0 = global_ns();
+                while (!mbar_try_wait(bars + L::B_KVFULL + s, (last_fill[s] / kStages) & 1) &&
+                       global_ns() - t0 < 100000000ull) {
+                }
+            }
+            if (tcount > 0) {
+                const uint64_t t0 = global_ns();
+                while (!mbar_try_wait(bars + L::B_QFULL, (tcount - 1) & 1) && global_ns() - t0 < 100000000ull) {
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ============================ MMA issuer ============================
+        constexpr uint32_t IDESC_QK = idesc_bf16_f32(kQ, kKV, false);
+        constexpr uint32_t IDESC_PV = idesc_bf16_f32(kQ, D, true);
+        const uint32_t q_addr = sbase + L::Q_OFF;
+        uint32_t fbase = 0;   // ring fill index of this tile's K_0 (K_j = fbase + 2j, V_j = +1)
+        int tcount = 0;
+        uint32_t p_use = 0;
+        bool ok = true;
+        for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
+            const TileInfo t = tile_info(p, idx);
+            if (!mbar_wait(bars + L::B_QFULL, tcount & 1, abort_flag, p.err)) break;
+            for (int j = 0; j < t.nkv && ok; ++j) {
+                // S_j = Q K_j^T
+                const uint32_t fk = fbase + 2 * (uint32_t)j;
+                const int kslot = fk % kStages;
+                if (!mbar_wait(bars + L::B_KVFULL + kslot, (fk / kStages) & 1, abort_flag, p.err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t k_addr = sbase + L::STAGE_OFF + kslot * L::TILE_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const int r = kk / 4, off = (kk % 4) * 32;
+                        const uint64_t adesc = sdesc_sw128(q_addr + r * L::REGION_BYTES + off, 16, 1024);
+                        const uint64_t bdesc = sdesc_sw128(k_addr + r * L::REGION_BYTES + off, 16, 1024);
+                        umma_ss(tmem + TM_S, adesc, bdesc, IDESC_QK, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(bars + L::B_KVEMPTY + kslot);
+                    umma_commit(bars + L::B_SFULL);
+                    if (j == t.nkv - 1) umma_commit(bars + L::B_QEMPTY);
+                }
+                __syncwarp();
+                // O += P_j V_j
+                if (!mbar_wait(bars + L::B_PFULL, p_use & 1, abort_flag, p.err)) {
+                    ok = false;
+                    break;
+                }
+                ++p_use;
+                const uint32_t fv = fk + 1;
+                const int vslot = fv % kStages;
+                if (!mbar_wait(bars + L::B_KVFULL + vslot, (fv / kStages) & 1, abort_flag, p.err)) {
+                    ok = false;
+                    break;
+                }
+                const int valid = min(kKV, t.lk - j * kKV);
+                if (valid < kKV) {
+                    // zero the V rows past the sequence (stale cache rows, or never loaded)
+                    uint8_t* vt = smem + L::STAGE_OFF + vslot * L::TILE_BYTES;
+                    for (int r = 0; r < L::REGIONS; ++r) {
+                        uint4* rowp = reinterpret_cast<uint4*>(vt + r * L::REGION_BYTES + valid * 128);
+                        const int n16 = (kKV - valid) * 8;
+                        for (int k = lane; k < n16; k += 32) rowp[k] = make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                if (j == 0 && tcount > 0) {
+                    if (!mbar_wait(bars + L::B_OFREE, (tcount - 1) & 1, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t v_addr = sbase + L::STAGE_OFF + vslot * L::TILE_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < kKV / 16; ++kk) {
+                        const uint64_t bdesc = sdesc_sw128(v_addr + kk * 16 * 128, L::REGION_BYTES, 1024);
+                        umma_ts(tmem + TM_O, tmem + TM_S + kk * 8, bdesc, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(bars + L::B_KVEMPTY + vslot);
+                    umma_commit(bars + L::B_ODONE);
+                    if (j == t.nkv - 1) umma_commit(bars + L::B_OFINAL);
+                }
+                __syncwarp();
+            }
+            fbase += 2 * (uint32_t)t.nkv;
+            ++tcount;
+        }
+        // every MMA this thread issued completes before TMEM is released
+        if (lane == 0) umma_commit(bars + L::B_DRAIN);
+        __syncwarp();
+        const uint64_t t0 = global_ns();
+        while (!mbar_try_wait(bars + L::B_DRAIN, 0) && global_ns() - t0 < 100000000ull) {
+        }
+    } else {
+        // ============================ softmax warps ============================
+        const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
+        const int r = quarter * 32 + lane;            // row of the tile: token r / P, head r % P
+        const int rtok = r >> p.pack_shift;
+        const int rhead = r & (p.pack - 1);
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        const uint32_t s_col = tmem + lane_base + TM_S;
+        const uint32_t o_col = tmem + lane_base + TM_O;
+        uint32_t s_use = 0;
+        int tcount = 0;
+        uint32_t pv_before = 0;                       // PVs issued for earlier tiles
+        for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
+            const TileInfo t = tile_info(p, idx);
+            const int pos = t.lk - t.lq + t.tok0 + rtok;           // absolute position of this row
+            const int lim = p.causal ? min(t.lk, pos + 1) : t.lk;  // keys 0 .. lim-1 are visible
+            const int lim_min = __reduce_min_sync(0xffffffffu, lim);
+            float m = -INFINITY, l = 0.f;
+            bool ok = true;
+            for (int j = 0; j < t.nkv; ++j) {
+                if (!mbar_wait(bars + L::B_SFULL, s_use & 1, abort_flag, p.err)) {
+                    ok = false;
+                    break;
+                }
+                ++s_use;
+                tc_fence_after();
+                const int key0 = j * kKV;
+                const bool open = key0 + kKV <= lim_min;          // no mask anywhere in the warp
+                // P_j against the current reference max, packed bf16 pairs in registers
+                uint32_t pk[kKV / 2];
+                float mt = -INFINITY, lt = 0.f;
+                const float m_use = m == -INFINITY ? INFINITY : m;   // first tile: all weights 0 for now
+#pragma unroll
+                for (int c = 0; c < kKV / 32; ++c) {
+                    uint32_t sv[32];
+                    tmem_ld32(s_col + c * 32, sv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int k = 0; k < 32; k += 2) {
+                        float x0 = __uint_as_float(sv[k]) * p.scale_log2;
+                        float x1 = __uint_as_float(sv[k + 1]) * p.scale_log2;
+                        if (!open) {
+                            x0 = (key0 + c * 32 + k < lim) ? x0 : -INFINITY;
+                            x1 = (key0 + c * 32 + k + 1 < lim) ? x1 : -INFINITY;
+                        }
+                        mt = fmaxf(mt, fmaxf(x0, x1));
+                        const float a = fast_exp2(x0 - m_use), b = fast_exp2(x1 - m_use);
+                        lt += a + b;
+                        pk[c * 16 + k / 2] = pack_bf16x2(a, b);
+                    }
+                }
+                const bool over = mt > m + kRescaleSlack;
+                if (__any_sync(0xffffffffu, over)) {
+                    const float m_new = over ? mt : m;
+                    const float alpha = over ? (m == -INFINITY ? 0.f : fast_exp2(m - m_new)) : 1.f;
+                    if (j > 0) {
+                        // O holds P_0..P_{j-1} V: wait for the last of them, then rescale
+                        if (!mbar_wait(bars + L::B_ODONE, (pv_before + j - 1) & 1, abort_flag, p.err)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+#pragma unroll
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t o[32];
+                            tmem_ld32(o_col + c * 32, o);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                            tmem_st32(o_col + c * 32, o);
+                        }
+                        tmem_wait_st();
+                    }
+                    l *= alpha;
+                    m = m_new;
+                    // recompute P_j against the new reference (S_j is still intact)
+                    const bool live = m > -INFINITY;
+                    lt = 0.f;
+#pragma unroll
+                    for (int c = 0; c < kKV / 32; ++c) {
+                        uint32_t sv[32];
+                        tmem_ld32(s_col + c * 32, sv);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int k = 0; k < 32; k += 2) {
+                            float x0 = __uint_as_float(sv[k]) * p.scale_log2;
+                            float x1 = __uint_as_float(sv[k + 1]) * p.scale_log2;
+                            x0 = (key0 + c * 32 + k < lim) ? x0 : -INFINITY;
+                            x1 = (key0 + c * 32 + k + 1 < lim) ? x1 : -INFINITY;
+                            const float a = live ? fast_exp2(x0 - m) : 0.f;
+                            const float b = live ? fast_exp2(x1 - m) : 0.f;
+                            lt += a + b;
+                            pk[c * 16 + k / 2] = pack_bf16x2(a, b);
+                        }
+                    }
+                }
+                l += lt;
+                tmem_st32(s_col, *reinterpret_cast<uint32_t(*)[32]>(pk));
+                tmem_st32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars + L::B_PFULL);
+            }
+            if (!ok) break;
+            if (!mbar_wait(bars + L::B_OFINAL, tcount & 1, abort_flag, p.err)) break;
+            tc_fence_after();
+            const bool row_ok = rtok < t.ntok;
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const size_t orow = (size_t)(t.q0 + t.tok0 + rtok) * p.hq + t.head0 + rhead;
+            uint4* dst = reinterpret_cast<uint4*>(p.out + orow * D);
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(o_col + c * 32, o);
+                tmem_wait_ld();
+                if (c == D / 32 - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bars + L::B_OFREE);
+                }
+                if (row_ok) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
+                        w.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
+                        w.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
+                        w.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
+                        dst[c * 4 + q] = w;
+                    }
+                }
+            }
+            if (row_ok && p.lse_out != nullptr) p.lse_out[orow] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+            pv_before += (uint32_t)t.nkv;
+            ++tcount;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 3-D view (dim, heads, rows) of a [rows, heads, dim] bf16 array; box = 64 x box_heads x
+// box_rows, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int dim, int heads, long long rows, int box_heads,
+              int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t gdim[3] = {(cuuint64_t)dim, (cuuint64_t)heads, (cuuint64_t)rows};
+    const cuuint64_t gstride[2] = {(cuuint64_t)dim * 2, (cuuint64_t)dim * heads * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
+    const cuuint32_t estride[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box, estride,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_prefill(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
+                           const PrefillParams& p, int grid, cudaStream_t stream) {
+    static std::once_flag once[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::call_once(once[dev & 63], [] {
+        cudaFuncSetAttribute(prefill_tcgen05_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Layout<D>::ALLOC);
+    });
+    prefill_tcgen05_kernel<D><<<grid, kThreads, Layout<D>::ALLOC, stream>>>(qm, km, vm, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t prefill_workspace_bytes(int batch, int total_q) {
+    const size_t entries = (size_t)std::max(0, batch) +
+                           ((size_t)std::max(0, total_q) + kMinTokensPerTile - 1) / kMinTokensPerTile;
+    return 256 + ((entries * sizeof(int2) + 255) & ~size_t(255));
+}
+
+nvpa_status_t run_varlen_prefill_tcgen05(const PrefillCall& c, void* workspace, size_t workspace_bytes,
+                                         cudaStream_t stream) {
+    const size_t need = prefill_workspace_bytes(c.batch, c.total_q);
+    if (workspace_bytes < need) {
+        set_error("workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+        return NVPA_ERR_WORKSPACE_TOO_SMALL;
+    }
+    // query heads packed per 128-row tile: the group size when it is a power of two <= 8
+    const int group = c.hq / c.hkv;
+    const int pack = (group & (group - 1)) == 0 ? std::min(group, kQ / kMinTokensPerTile) : 1;
+    CUtensorMap qm, km, vm;
+    const int box_kv = std::min(c.block_size, kKV);
+    if (!make_map(&qm, c.q, c.head_dim, c.hq, c.total_q, pack, kQ / pack) ||
+        !make_map(&km, c.k_cache, c.head_dim, c.hkv, (long long)c.num_blocks * c.block_size, 1, box_kv) ||
+        !make_map(&vm, c.v_cache, c.head_dim, c.hkv, (long long)c.num_blocks * c.block_size, 1, box_kv)) {
+        set_error("cuTensorMapEncodeTiled failed (driver entry point missing or bad layout)");
+        return NVPA_ERR_CUDA;
+    }
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    PrefillParams p{};
+    p.block_tables = c.block_tables;
+    p.cu_q = c.cu_seqlens_q;
+    p.cu_k = c.cu_seqlens_k;
+    p.out = static_cast<uint16_t*>(c.out);
+    p.lse_out = c.lse_out;
+    p.err = c.err_flag;
+    p.ntiles = reinterpret_cast<int32_t*>(ws);
+    p.tiles = reinterpret_cast<int2*>(ws + 256);
+    p.batch = c.batch;
+    p.total_q = c.total_q;
+    p.hq = c.hq;
+    p.hkv = c.hkv;
+    p.group = group;
+    p.pack = pack;
+    p.pack_shift = __builtin_ctz((unsigned)pack);
+    p.tq = kQ / pack;
+    p.hgroups = c.hq / pack;
+    p.max_blocks = c.max_blocks_per_seq;
+    p.num_blocks = c.num_blocks;
+    p.block_size = c.block_size;
+    p.block_shift = __builtin_ctz((unsigned)c.block_size);
+    p.max_q = c.max_seqlen_q;
+    p.max_k = c.max_seqlen_k;
+    p.causal = c.causal;
+    p.scale_log2 = c.scale * kLog2e;
+
+    prefill_plan_kernel<<<1, 1024, 0, stream>>>(p, reinterpret_cast<int2*>(ws + 256), reinterpret_cast<int32_t*>(ws));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_failure(e, "prefill plan launch");
+    count_launches(1);
+    const long long max_tiles = ((long long)c.batch + (c.total_q + p.tq - 1) / p.tq) * p.hgroups;
+    const int grid = (int)std::max(1LL, std::min<long long>(2LL * device_sm_count(), max_tiles));
+    e = c.head_dim == 128 ? launch_prefill<128>(qm, km, vm, p, grid, stream)
+                          : launch_prefill<64>(qm, km, vm, p, grid, stream);
+    if (e != cudaSuccess) return cuda_failure(e, "prefill tcgen05 launch");
+    count_launches(1);
+    return NVPA_OK;
+}
+
+}  // namespace nvpa

@@ -102,17 +102,20 @@ def test_store_host_checks(lib):
 def test_prefill_host_checks(lib):
     def pf(**kw):
         a = dict(batch=2, total_q=10, mq=8, mk=8, hq=4, hkv=2, d=64, nb=8, bs=16, causal=1,
-                 q=FAKE)
+                 q=FAKE, ws=FAKE)
         a.update(kw)
         return lib.nvpa_varlen_prefill_attention(FAKE, None, a["q"], FAKE, FAKE, FAKE, 2, FAKE,
                                                  FAKE, a["batch"], a["total_q"], a["mq"], a["mk"],
                                                  a["hq"], a["hkv"], a["d"], a["nb"], a["bs"], 0.1,
-                                                 a["causal"], None, None)
+                                                 a["causal"], a["ws"], 1 << 20, None, None)
     assert pf(causal=2) == _lib.NVPA_ERR_INVALID_ARG
     assert pf(d=256) == _lib.NVPA_ERR_UNSUPPORTED
     assert pf(total_q=0) == _lib.NVPA_OK
     assert pf(q=None) == _lib.NVPA_ERR_INVALID_ARG
     assert pf(total_q=-3) == _lib.NVPA_ERR_INVALID_ARG
+    assert pf(ws=None) == _lib.NVPA_ERR_INVALID_ARG
+    assert pf(ws=FAKE + 64) == _lib.NVPA_ERR_INVALID_ARG
+    assert lib.nvpa_varlen_prefill_workspace_size(32, 24594) >= 8 * (32 + 24594 // 128)
 
 
 def test_gather_host_checks(lib):
