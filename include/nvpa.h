@@ -175,6 +175,35 @@ nvpa_status_t nvpa_paged_decode_attention(void* out, float* lse_out, const void*
                                           int32_t* err_flag, cudaStream_t stream);
 
 /*
+ * nvpa_decode_step -- one decode step in one call: store each sequence's new key/value
+ * row and attend over the context that includes it ([P1] 5.2: decode prepares one token
+ * per sequence with its slot mapping; [P3] store_kvcache then flash_attn_with_kvcache).
+ * Equivalent to nvpa_store_kvcache(k_new, v_new, ..., slot_mapping, batch) followed by
+ * nvpa_paged_decode_attention(...), under the decode contract that sequence b's new
+ * token is its key at position context_lens[b] - 1 and slot_mapping[b] is that
+ * position's cache slot (-1: not stored, e.g. a padded batch entry).  The attention reads
+ * the new row from k_new/v_new directly and the row is written to the cache from the
+ * kernel that consumes it, so there is no separate store launch and no read-after-write
+ * through the cache.
+ *
+ *   k_new, v_new    bf16 [batch, num_kv_heads, head_dim] with token strides as in
+ *                   nvpa_store_kvcache.
+ *   slot_mapping    int32 [batch].  Out-of-range slots other than -1 set
+ *                   NVPA_FLAG_BAD_SLOT and are not written.
+ *   other arguments as for nvpa_paged_decode_attention (same workspace size).
+ */
+nvpa_status_t nvpa_decode_step(void* out, float* lse_out, const void* q,
+                               const void* k_new, const void* v_new,
+                               int64_t k_token_stride, int64_t v_token_stride,
+                               void* k_cache, void* v_cache, const int32_t* slot_mapping,
+                               const int32_t* block_tables, int max_blocks_per_seq,
+                               const int32_t* context_lens, int batch, int num_q_heads,
+                               int num_kv_heads, int head_dim, int num_blocks, int block_size,
+                               int max_context_len, float softmax_scale, int num_splits,
+                               void* workspace, size_t workspace_bytes, int32_t* err_flag,
+                               cudaStream_t stream);
+
+/*
  * nvpa_paged_decode_attention_static_scratch -- the same decode attention for callers
  * that cannot allocate device memory: a plugin inside a host runtime whose memory
  * manager owns all device memory and offers no allocation hook, or code running where an

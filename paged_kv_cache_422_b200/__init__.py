@@ -15,6 +15,7 @@ from ._lib import (  # noqa: F401
     lib,
 )
 from .api import (  # noqa: F401
+    decode_step,
     gather_kv,
     paged_decode_attention,
     paged_decode_workspace_size,

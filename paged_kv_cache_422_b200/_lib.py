@@ -37,6 +37,8 @@ SIGNATURES = {
     "nvpa_paged_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "nvpa_paged_decode_attention": (_i, [_p, _p, _p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i,
                                          _i, _f, _i, _p, _sz, _p, _p]),
+    "nvpa_decode_step": (_i, [_p, _p, _p, _p, _p, _i64, _i64, _p, _p, _p, _p, _i, _p, _i, _i, _i,
+                              _i, _i, _i, _i, _f, _i, _p, _sz, _p, _p]),
     "nvpa_paged_decode_attention_static_scratch": (_i, [_p, _p, _p, _p, _p, _p, _i, _p, _i, _i,
                                                         _i, _i, _i, _i, _i, _f, _i, _p, _p]),
     "nvpa_varlen_prefill_workspace_size": (_sz, [_i, _i]),

@@ -114,6 +114,42 @@ def paged_decode_attention(q, k_cache, v_cache, block_tables, context_lens, max_
     return (out, lse) if return_lse else out
 
 
+def decode_step(q, k_new, v_new, k_cache, v_cache, slot_mapping, block_tables, context_lens,
+                max_context_len, softmax_scale, out=None, lse=None, workspace=None, num_splits=0,
+                err_flag=None, stream=None, return_lse=False):
+    """Store each sequence's new K/V row (k_new[b] -> slot_mapping[b]) and run decode
+    attention over contexts that include it, in one call."""
+    nb, bs, hkv, d = _cache_dims(k_cache, v_cache)
+    _need(q, _BF16, "q", 3)
+    _contig(q, "q")
+    b, hq, dq = (int(x) for x in q.shape)
+    if dq != d:
+        raise ValueError("q head_dim differs from the cache's")
+    for name, t in (("k_new", k_new), ("v_new", v_new)):
+        _need(t, _BF16, name, 3)
+        if tuple(t.shape) != (b, hkv, d) or t.stride(2) != 1 or t.stride(1) != d:
+            raise ValueError(f"{name} must be [{b}, {hkv}, {d}] with contiguous heads and dims")
+    for name, t in (("slot_mapping", slot_mapping), ("block_tables", block_tables),
+                    ("context_lens", context_lens)):
+        _need(t, _I32, name)
+        _contig(t, name)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((b, hq), dtype=torch.float32, device=q.device)
+    need = paged_decode_workspace_size(b, hq, hkv, d, max_context_len, bs, num_splits)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = lib().nvpa_decode_step(
+        _ptr(out), _ptr(lse), _ptr(q), _ptr(k_new), _ptr(v_new), k_new.stride(0), v_new.stride(0),
+        _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), _ptr(block_tables),
+        int(block_tables.shape[1]), _ptr(context_lens), b, hq, hkv, d, nb, bs,
+        int(max_context_len), float(softmax_scale), int(num_splits), _ptr(workspace),
+        int(workspace.numel() * workspace.element_size()), _ptr(err_flag), _stream_handle(stream))
+    check(st, "nvpa_decode_step")
+    return (out, lse) if return_lse else out
+
+
 def varlen_prefill_workspace_size(batch, total_q) -> int:
     return int(lib().nvpa_varlen_prefill_workspace_size(batch, total_q))
 

@@ -31,6 +31,11 @@ struct DecodeCall {
     void* workspace;
     size_t workspace_bytes;
     int32_t* err_flag;
+    // fused decode step (nvpa_decode_step); k_new == nullptr for plain decode
+    const void* k_new = nullptr;
+    const void* v_new = nullptr;
+    long long k_new_stride = 0, v_new_stride = 0;
+    const int32_t* slot_mapping = nullptr;
 };
 
 struct PrefillCall {

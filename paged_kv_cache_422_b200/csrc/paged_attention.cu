@@ -40,6 +40,16 @@ struct AttnParams {
     const uint16_t* v_cache;
     const int32_t* block_tables;
     const int32_t* context_lens;
+    // fused decode step: sequence b's newest key/value (position context_lens[b]-1) is read
+    // from k_new/v_new row b instead of the cache and written to slot_mapping[b]
+    const uint16_t* k_new;
+    const uint16_t* v_new;
+    long long k_new_stride, v_new_stride;   // elements between rows of k_new / v_new
+    const int32_t* slot_mapping;
+    long long capacity;                     // num_blocks * block_size
+    int fused;
+    uint16_t* k_cache_w;
+    uint16_t* v_cache_w;
     uint16_t* out;
     float* lse_out;
     float* o_part;
@@ -59,8 +69,15 @@ template <int D, int GMAX>
 struct AttnStage {
     static constexpr int KV_BYTES = kTileKeys * D * 2;
     static constexpr int Q_BYTES = GMAX * D * 2;
-    static constexpr int BYTES = 2 * KV_BYTES + Q_BYTES + 16;
+    static constexpr int BYTES = 2 * KV_BYTES + Q_BYTES + 32;   // + two int4 of metadata
 };
+
+// Programmatic dependent launch: wait for the preceding kernel's results / let the next
+// kernel's CTAs start launching.  Both are no-ops for a normal launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 // ------------------------------------------------------------------------------------
 // plan: context lengths -> (sequence, partition, key range) table
@@ -69,6 +86,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const AttnParams p) {
     __shared__ int warp_tot[32];
     __shared__ int carry_s;
     const int tid = threadIdx.x;
+    pdl_launch_dependents();
     const int lane = tid & 31, wid = tid >> 5;
     if (tid == 0) carry_s = 0;
     __syncthreads();
@@ -142,6 +160,7 @@ paged_attention_kernel(const AttnParams p) {
     int it_ntiles = 0, it_t = 0, it_fb = 0, it_blk = -1;
     const int32_t* it_bt = nullptr;
 
+    pdl_wait();   // the plan (and everything before it on the stream) has completed
     // Lane 0 holds the next item index, requested one item ahead.
     const int total_items = __ldcg(p.counter + 1);
     int nx_item = 0;
@@ -188,7 +207,7 @@ paged_attention_kernel(const AttnParams p) {
         ks = reinterpret_cast<uint16_t*>(sb);
         vs = ks + kTileKeys * D;
         qs = vs + kTileKeys * D;
-        meta = reinterpret_cast<int4*>(qs + GMAX * D);
+        meta = reinterpret_cast<int4*>(qs + GMAX * D);   // meta[0], meta[1]
     };
 
     auto issue = [&](int st) {
@@ -216,22 +235,33 @@ paged_attention_kernel(const AttnParams p) {
         const size_t slot0 = (size_t)max(blk, 0) * p.block_size + (key0 & bmask);
         const uint16_t* kg = p.k_cache + slot0 * row_stride + (size_t)it_hk * D + sub * 8;
         const uint16_t* vg = p.v_cache + slot0 * row_stride + (size_t)it_hk * D + sub * 8;
+        const bool first = it_t == 0;
+        const bool last = it_t + 1 == it_ntiles;
+        // fused step: the sequence's newest key sits in the last tile of its last partition
+        const int new_row = (p.fused && last && it_s + 1 == it_ns && it_k1 > key0) ? it_k1 - 1 - key0 : -1;
 #pragma unroll
         for (int i = 0; i < ITER; ++i) {
             const int r = grp + RPI * i;
             const int nb = r < rows ? 16 : 0;
-            cp_async16(ks + r * D + sub * 8, kg + (size_t)r * row_stride, nb);
-            cp_async16(vs + r * D + sub * 8, vg + (size_t)r * row_stride, nb);
+            if (r == new_row) {
+                cp_async16(ks + r * D + sub * 8,
+                           p.k_new + (size_t)it_seq * p.k_new_stride + (size_t)it_hk * D + sub * 8, 16);
+                cp_async16(vs + r * D + sub * 8,
+                           p.v_new + (size_t)it_seq * p.v_new_stride + (size_t)it_hk * D + sub * 8, 16);
+            } else {
+                cp_async16(ks + r * D + sub * 8, kg + (size_t)r * row_stride, nb);
+                cp_async16(vs + r * D + sub * 8, vg + (size_t)r * row_stride, nb);
+            }
         }
-        const bool first = it_t == 0;
-        const bool last = it_t + 1 == it_ntiles;
         if (first) {
             const uint16_t* qg = p.q + ((size_t)it_qrow * p.hq + (size_t)it_hk * p.group) * D;
             for (int c = lane; c < p.group * LPR; c += 32) cp_async16(qs + c * 8, qg + c * 8, 16);
         }
-        if (lane == 0)
-            *meta = make_int4(it_qrow, it_hk, it_s | (it_ns << 16),
-                              rows | (first ? 256 : 0) | (last ? 512 : 0));
+        if (lane == 0) {
+            meta[0] = make_int4(it_qrow, it_hk, it_s | (it_ns << 16),
+                                rows | (first ? 256 : 0) | (last ? 512 : 0));
+            meta[1] = make_int4(new_row, new_row >= 0 ? __ldg(p.slot_mapping + it_seq) : -1, 0, 0);
+        }
         cp_async_commit();
         if (last) fetch(); else ++it_t;
     };
@@ -280,6 +310,21 @@ paged_attention_kernel(const AttnParams p) {
             acc.load_q(qs, p.group, sub, p.scale_log2);
         }
         acc.consume(ks, vs, rows, lane);
+        if (p.fused) {
+            const int4 m1 = meta_p[1];
+            if (m1.x >= 0 && grp == (m1.x % RPI)) {
+                const int slot = m1.y;
+                if (slot >= 0 && (long long)slot < p.capacity) {
+                    const size_t dst = (size_t)slot * row_stride + (size_t)meta.y * D + sub * 8;
+                    *reinterpret_cast<uint4*>(p.k_cache_w + dst) =
+                        *reinterpret_cast<const uint4*>(ks + m1.x * D + sub * 8);
+                    *reinterpret_cast<uint4*>(p.v_cache_w + dst) =
+                        *reinterpret_cast<const uint4*>(vs + m1.x * D + sub * 8);
+                } else if (slot != -1 && sub == 0) {
+                    flag_error(p.err, NVPA_FLAG_BAD_SLOT);
+                }
+            }
+        }
         if (meta.w & 512) epilogue(meta);
         return true;
     };
@@ -297,6 +342,7 @@ paged_attention_kernel(const AttnParams p) {
         cs = (cs + 1 == STAGES) ? 0 : cs + 1;
     }
     cp_async_wait<0>();
+    pdl_launch_dependents();
 }
 
 // ------------------------------------------------------------------------------------
@@ -305,6 +351,7 @@ paged_attention_kernel(const AttnParams p) {
 template <int D>
 __global__ void __launch_bounds__(256) decode_combine_kernel(const AttnParams p) {
     constexpr int DPL = D / 32;   // output dims per lane
+    pdl_wait();
     const int w = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (w >= p.batch * p.hq) return;
@@ -373,6 +420,24 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const AttnParams p)
 // ------------------------------------------------------------------------------------
 namespace {
 
+// Launch with programmatic stream serialisation: the kernel may start while its
+// predecessor finishes and synchronises with it through griddepcontrol.wait.
+template <typename Kernel>
+cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       const AttnParams& p) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 template <int D, int GMAX>
 int worker_ctas_per_sm() {
     static std::once_flag once[64];
@@ -398,8 +463,8 @@ cudaError_t launch_worker(const AttnParams& p, long long max_items, cudaStream_t
     const long long want = (max_items + kAttnWarps - 1) / kAttnWarps;
     const int grid = (int)std::max(1LL, std::min<long long>((long long)device_sm_count() * per_sm, want));
     const int smem = kAttnWarps * kAttnStages * AttnStage<D, GMAX>::BYTES;
-    paged_attention_kernel<D, GMAX><<<grid, kAttnWarps * 32, smem, stream>>>(p);
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = launch_pdl(paged_attention_kernel<D, GMAX>, dim3(grid), dim3(kAttnWarps * 32),
+                                     (size_t)smem, stream, p);
     if (e == cudaSuccess) count_launches(1);
     return e;
 }
@@ -492,6 +557,15 @@ nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream) {
     p.chunk = chunk;
     p.s_max = s_max;
     p.scale_log2 = c.scale * kLog2e;
+    p.fused = c.k_new != nullptr ? 1 : 0;
+    p.k_new = static_cast<const uint16_t*>(c.k_new);
+    p.v_new = static_cast<const uint16_t*>(c.v_new);
+    p.k_new_stride = c.k_new_stride;
+    p.v_new_stride = c.v_new_stride;
+    p.slot_mapping = c.slot_mapping;
+    p.capacity = (long long)c.num_blocks * c.block_size;
+    p.k_cache_w = static_cast<uint16_t*>(const_cast<void*>(c.k_cache));
+    p.v_cache_w = static_cast<uint16_t*>(const_cast<void*>(c.v_cache));
 
     decode_plan_kernel<<<1, 1024, 0, stream>>>(p);
     cudaError_t e = cudaGetLastError();
@@ -503,9 +577,8 @@ nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream) {
     if (s_max > 1) {
         const long long warps = (long long)c.batch * c.hq;
         const int grid = (int)((warps + 7) / 8);
-        if (c.head_dim == 128) decode_combine_kernel<128><<<grid, 256, 0, stream>>>(p);
-        else decode_combine_kernel<64><<<grid, 256, 0, stream>>>(p);
-        e = cudaGetLastError();
+        e = c.head_dim == 128 ? launch_pdl(decode_combine_kernel<128>, dim3(grid), dim3(256), 0, stream, p)
+                              : launch_pdl(decode_combine_kernel<64>, dim3(grid), dim3(256), 0, stream, p);
         if (e != cudaSuccess) return cuda_failure(e, "decode combine launch");
         count_launches(1);
     }

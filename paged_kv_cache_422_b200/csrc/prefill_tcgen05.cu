@@ -122,15 +122,18 @@ __device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, int idx) {
 // ------------------------------------------------------------------------------------
 // plan: list (sequence, query tile) pairs, most key tiles first
 // ------------------------------------------------------------------------------------
-constexpr int kPlanBins = 1024;
+constexpr int kPlanMaxRanked = 2048;   // batches up to this size are ordered by sequence
 
+// Entries are grouped by sequence, sequences with the most work (key tiles visited over
+// all their query tiles) first and, inside a sequence, query tiles with the most key
+// tiles first.  CTAs that run at the same time then mostly read the same sequences' keys
+// and values, which L2 serves after the first fetch, and the longest work starts first.
 __global__ void __launch_bounds__(1024) prefill_plan_kernel(const PrefillParams p, int2* tiles,
                                                             int32_t* ntiles) {
-    __shared__ int hist[kPlanBins];
-    __shared__ int cursor[kPlanBins];
-    const int tid = threadIdx.x;
-    for (int i = tid; i < kPlanBins; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
+    __shared__ int s_work[kPlanMaxRanked];
+    __shared__ int s_count[kPlanMaxRanked];
+    __shared__ int warp_tot[32];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const long long cap = (long long)p.max_blocks * p.block_size;
     auto seq_ok = [&](int i, int& lq, int& lk) {
         const int q0 = __ldg(p.cu_q + i), q1 = __ldg(p.cu_q + i + 1);
@@ -140,36 +143,103 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const PrefillParams 
         return q0 >= 0 && lq >= 0 && lk >= lq && lq <= p.max_q && lk <= p.max_k && lk <= cap &&
                q1 <= p.total_q;
     };
-    auto nkv_of = [&](int lq, int lk, int qt) {
-        const int tok0 = qt * p.tq;
-        return min(max(tile_nkv(p.causal, lq, lk, tok0, min(p.tq, lq - tok0)), 0), kPlanBins - 1);
-    };
-    for (int i = tid; i < p.batch; i += blockDim.x) {
-        int lq, lk;
-        if (!seq_ok(i, lq, lk)) {
-            flag_error(p.err, NVPA_FLAG_BAD_LENGTH);
-            continue;
+    const int nb = min(p.batch, kPlanMaxRanked);
+    // per sequence: tiles and work (0 tiles for a malformed sequence, which is flagged)
+    for (int i = tid; i < kPlanMaxRanked; i += blockDim.x) {
+        int lq = 0, lk = 0, cnt = 0, work = 0;
+        if (i < p.batch) {
+            if (seq_ok(i, lq, lk)) {
+                cnt = (lq + p.tq - 1) / p.tq;
+                for (int qt = 0; qt < cnt; ++qt)
+                    work += tile_nkv(p.causal, lq, lk, qt * p.tq, min(p.tq, lq - qt * p.tq));
+            } else {
+                flag_error(p.err, NVPA_FLAG_BAD_LENGTH);
+            }
         }
-        for (int qt = 0; qt * p.tq < lq; ++qt) atomicAdd(&hist[nkv_of(lq, lk, qt)], 1);
+        if (i < nb) {
+            s_work[i] = work;
+            s_count[i] = cnt;
+        }
     }
     __syncthreads();
-    if (tid == 0) {   // descending prefix: most key tiles first
-        int acc = 0;
-        for (int b = kPlanBins - 1; b >= 0; --b) {
-            cursor[b] = acc;
-            acc += hist[b];
+    // rank of each of the first nb sequences: heavier first, ties by index
+    int rank_of[kPlanMaxRanked / 1024];
+    for (int k = 0; k < kPlanMaxRanked / 1024; ++k) {
+        const int i = tid + k * 1024;
+        int rnk = 0;
+        if (i < nb) {
+            const int wi = s_work[i];
+            for (int jj = 0; jj < nb; ++jj) {
+                const int wj = s_work[jj];
+                rnk += (wj > wi || (wj == wi && jj < i)) ? 1 : 0;
+            }
         }
-        *ntiles = acc;
+        rank_of[k] = rnk;
     }
     __syncthreads();
-    for (int i = tid; i < p.batch; i += blockDim.x) {
+    // reorder the tile counts by rank (reuse s_work as counts-in-rank-order)
+    for (int k = 0; k < kPlanMaxRanked / 1024; ++k) {
+        const int i = tid + k * 1024;
+        if (i < nb) s_work[rank_of[k]] = s_count[i];
+    }
+    __syncthreads();
+    // exclusive prefix over ranks (two 1024-element passes)
+    int carry = 0;
+    for (int k = 0; k < kPlanMaxRanked / 1024; ++k) {
+        const int r = tid + k * 1024;
+        int v = r < nb ? s_work[r] : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
+        }
+        if (lane == 31) warp_tot[wid] = incl;
+        __syncthreads();
+        if (wid == 0) {
+            int w = warp_tot[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += n;
+            }
+            warp_tot[lane] = w;
+        }
+        __syncthreads();
+        const int excl = carry + incl - v + (wid ? warp_tot[wid - 1] : 0);
+        const int block_total = warp_tot[31];
+        __syncthreads();
+        if (r < nb) s_count[r] = excl;   // s_count now: offset of rank r
+        carry += block_total;
+    }
+    __syncthreads();
+    int written = carry;
+    // write each ranked sequence's tiles, most key tiles (last query tile) first
+    for (int k = 0; k < kPlanMaxRanked / 1024; ++k) {
+        const int i = tid + k * 1024;
+        if (i >= nb) continue;
         int lq, lk;
         if (!seq_ok(i, lq, lk)) continue;
-        for (int qt = 0; qt * p.tq < lq; ++qt) {
-            const int pos = atomicAdd(&cursor[nkv_of(lq, lk, qt)], 1);
-            tiles[pos] = make_int2(i, qt);
-        }
+        const int cnt = (lq + p.tq - 1) / p.tq;
+        const int off = s_count[rank_of[k]];
+        for (int u = 0; u < cnt; ++u) tiles[off + u] = make_int2(i, cnt - 1 - u);
     }
+    // sequences beyond the ranked ones (very large batches) follow in index order
+    if (p.batch > nb) {
+        __shared__ int extra_base;
+        if (tid == 0) extra_base = written;
+        __syncthreads();
+        for (int i = nb + tid; i < p.batch; i += blockDim.x) {
+            int lq, lk;
+            if (!seq_ok(i, lq, lk)) continue;
+            const int cnt = (lq + p.tq - 1) / p.tq;
+            const int off = atomicAdd(&extra_base, cnt);
+            for (int u = 0; u < cnt; ++u) tiles[off + u] = make_int2(i, cnt - 1 - u);
+        }
+        __syncthreads();
+        if (tid == 0) written = extra_base;
+    }
+    if (tid == 0) *ntiles = written;
 }
 
 // ------------------------------------------------------------------------------------
@@ -224,63 +294,74 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
 
     if (warp == 0) {
         // ============================ TMA producer ============================
-        if (lane == 0) {
-            uint32_t fill = 0;
-            int tcount = 0;
-            int last_fill[kStages];
-            for (int s = 0; s < kStages; ++s) last_fill[s] = -1;
-            for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
-                const TileInfo t = tile_info(p, idx);
-                if (!mbar_wait(bars + L::B_QEMPTY, (tcount & 1) ^ 1, abort_flag, p.err)) break;
+        // The whole warp walks the tiles; lane 0 issues the copies and barrier operations,
+        // lane c < 8 holds the physical block of piece c of the next key tile, loaded one
+        // key tile ahead so that no copy waits on a block-table lookup.
+        uint32_t fill = 0;
+        int tcount = 0;
+        int last_fill[kStages];
+        for (int s = 0; s < kStages; ++s) last_fill[s] = -1;
+        const int piece = min(p.block_size, kKV);
+        auto load_pieces = [&](const int32_t* bt, int lk, int j) {
+            const int key0 = j * kKV;
+            const int npieces = (min(kKV, lk - key0) + piece - 1) / piece;
+            int blk = -1;
+            if (lane < npieces) {
+                blk = __ldg(bt + ((key0 + lane * piece) >> p.block_shift));
+                if (blk < 0 || blk >= p.num_blocks) {
+                    flag_error(p.err, NVPA_FLAG_BAD_BLOCK_ID);
+                    blk = -1;
+                }
+            }
+            return blk;
+        };
+        for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
+            const TileInfo t = tile_info(p, idx);
+            const int32_t* bt = p.block_tables + (size_t)t.seq * p.max_blocks;
+            int cur_blk = load_pieces(bt, t.lk, 0);
+            if (!mbar_wait(bars + L::B_QEMPTY, (tcount & 1) ^ 1, abort_flag, p.err)) break;
+            if (lane == 0) {
                 mbar_arrive_expect_tx(bars + L::B_QFULL, L::TILE_BYTES);
                 for (int r = 0; r < L::REGIONS; ++r)
                     tma_load_3d(smem + L::Q_OFF + r * L::REGION_BYTES, &q_map, bars + L::B_QFULL, r * 64,
                                 t.head0, t.q0 + t.tok0);
-                const int32_t* bt = p.block_tables + (size_t)t.seq * p.max_blocks;
-                const int piece = min(p.block_size, kKV);
-                bool ok = true;
-                for (int j = 0; j < t.nkv && ok; ++j) {
-                    const int key0 = j * kKV;
-                    const int nrows = min(kKV, t.lk - key0);
-                    const int npieces = (nrows + piece - 1) / piece;
-                    for (int kv = 0; kv < 2; ++kv) {
-                        const int slot = fill % kStages;
-                        if (!mbar_wait(bars + L::B_KVEMPTY + slot, ((fill / kStages) & 1) ^ 1, abort_flag, p.err)) {
-                            ok = false;
-                            break;
-                        }
-                        uint8_t* dst = smem + L::STAGE_OFF + slot * L::TILE_BYTES;
-                        uint32_t bytes = 0;
-                        int blks[kKV / 16];
-                        for (int c = 0; c < npieces; ++c) {
+            }
+            bool ok = true;
+            for (int j = 0; j < t.nkv && ok; ++j) {
+                const int nxt_blk = j + 1 < t.nkv ? load_pieces(bt, t.lk, j + 1) : -1;
+                const int key0 = j * kKV;
+                const uint32_t valid_mask = __ballot_sync(0xffffffffu, cur_blk >= 0);
+                const uint32_t bytes = (uint32_t)__popc(valid_mask) * (uint32_t)(piece * 128 * L::REGIONS);
+                for (int kv = 0; kv < 2; ++kv) {
+                    const int slot = fill % kStages;
+                    if (!mbar_wait(bars + L::B_KVEMPTY + slot, ((fill / kStages) & 1) ^ 1, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* dst = smem + L::STAGE_OFF + slot * L::TILE_BYTES;
+                    const CUtensorMap* map = kv ? &v_map : &k_map;
+                    if (lane == 0) mbar_arrive_expect_tx(bars + L::B_KVFULL + slot, bytes);
+                    for (uint32_t m = valid_mask; m != 0; m &= m - 1) {
+                        const int c = __ffs(m) - 1;
+                        const int blk = __shfl_sync(0xffffffffu, cur_blk, c);
+                        if (lane == 0) {
                             const int kc = key0 + c * piece;
-                            int blk = __ldg(bt + (kc >> p.block_shift));
-                            if (blk < 0 || blk >= p.num_blocks) {
-                                flag_error(p.err, NVPA_FLAG_BAD_BLOCK_ID);
-                                blk = -1;
-                            } else {
-                                bytes += (uint32_t)(piece * 128 * L::REGIONS);
-                            }
-                            blks[c] = blk;
-                        }
-                        mbar_arrive_expect_tx(bars + L::B_KVFULL + slot, bytes);
-                        const CUtensorMap* map = kv ? &v_map : &k_map;
-                        for (int c = 0; c < npieces; ++c) {
-                            if (blks[c] < 0) continue;
-                            const int kc = key0 + c * piece;
-                            const int z = blks[c] * p.block_size + (kc & (p.block_size - 1));
+                            const int z = blk * p.block_size + (kc & (p.block_size - 1));
                             for (int r = 0; r < L::REGIONS; ++r)
                                 tma_load_3d(dst + r * L::REGION_BYTES + c * piece * 128, map,
                                             bars + L::B_KVFULL + slot, r * 64, t.hk, z);
                         }
-                        last_fill[slot] = (int)fill;
-                        ++fill;
                     }
+                    last_fill[slot] = (int)fill;
+                    ++fill;
                 }
-                ++tcount;
-                if (!ok) break;
+                cur_blk = nxt_blk;
             }
-            // let every copy this thread started land before the CTA can exit
+            ++tcount;
+            if (!ok) break;
+        }
+        // let every copy this warp started land before the CTA can exit
+        if (lane == 0) {
             for (int s = 0; s < kStages; ++s) {
                 if (last_fill[s] < 0) continue;
                 const uint64_t t0 = global_ns();
