@@ -4,7 +4,9 @@ Default workload: one decode step at batch 512 with prefix sharing (lognormal co
 lengths, median 1024, clipped to [16, 4096]; half the sequences share a 1024-token prefix
 held in 4 physical blocks; 16 query / 8 KV heads, head_dim 128, block size 256, bf16).
 A step stores the 512 new tokens' K/V rows and runs paged decode attention over the
-contexts that include them (one nvpa_decode_step call).
+contexts that include them, in one call: nvpa_decode_step_shared_prefix by default (the
+shared prefix is attended once for its group on the tensor cores), nvpa_decode_step with
+--decode-api plain.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl nvpa|reference]
                     [--workload NAME]
@@ -177,7 +179,9 @@ def profile_traffic(kernel_tag: str, source_files) -> float | None:
 
 DECODE_SOURCES = ["paged_kv_cache_422_b200/csrc/paged_attention.cu",
                   "paged_kv_cache_422_b200/csrc/attn_warp.cuh",
-                  "paged_kv_cache_422_b200/csrc/common.cuh"]
+                  "paged_kv_cache_422_b200/csrc/common.cuh",
+                  "paged_kv_cache_422_b200/csrc/prefill_tcgen05.cu",
+                  "paged_kv_cache_422_b200/csrc/sm100.cuh"]
 
 
 def source_sha(files) -> str:
@@ -327,20 +331,27 @@ def run_nvpa(args) -> int:
     work = decode_step_bytes(step)
     t = decode_to_device(step, dev)
     stream = torch.cuda.Stream(device=dev)
-    ws_bytes = nvpa.paged_decode_workspace_size(step.batch, step.num_q_heads, step.num_kv_heads,
-                                                step.head_dim, step.max_context_len,
-                                                step.block_size, args.num_splits)
+    shared = args.decode_api == "shared"
+    if shared:
+        ws_bytes = nvpa.decode_shared_prefix_workspace_size(
+            step.batch, step.num_q_heads, step.num_kv_heads, step.head_dim, step.max_context_len,
+            step.block_size, args.num_splits)
+    else:
+        ws_bytes = nvpa.paged_decode_workspace_size(
+            step.batch, step.num_q_heads, step.num_kv_heads, step.head_dim, step.max_context_len,
+            step.block_size, args.num_splits)
     workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     out = torch.empty_like(t["q"])
+    decode_call = nvpa.decode_step_shared_prefix if shared else nvpa.decode_step
 
     def one_step(ev=None):
         # store + decode in one call (the library's fused decode step)
         if ev is not None:
             ev[0].record(stream)
-        nvpa.decode_step(t["q"], t["k_new"], t["v_new"], t["k_cache"], t["v_cache"],
-                         t["slot_mapping"], t["block_tables"], t["context_lens"],
-                         step.max_context_len, step.scale, out=out, workspace=workspace,
-                         num_splits=args.num_splits, stream=stream)
+        decode_call(t["q"], t["k_new"], t["v_new"], t["k_cache"], t["v_cache"],
+                    t["slot_mapping"], t["block_tables"], t["context_lens"],
+                    step.max_context_len, step.scale, out=out, workspace=workspace,
+                    num_splits=args.num_splits, stream=stream)
         if ev is not None:
             ev[1].record(stream)
 
@@ -416,8 +427,12 @@ def run_nvpa(args) -> int:
                     parallelism=f"replicas x{world}" if world > 1 else "single GPU",
                     l2="inputs larger than L2: %.2f GB of unique K/V per step vs 126 MB L2"
                        % (work["kv_unique"] / 1e9),
-                    num_splits=args.num_splits),
-        roofline=dict(bound="hbm", kernel="decode_step (plan + split-KV worker with the store folded in + combine)",
+                    num_splits=args.num_splits,
+                    decode_api=("nvpa_decode_step_shared_prefix" if shared else "nvpa_decode_step")),
+        roofline=dict(bound="hbm",
+                      kernel=("decode step: plan, shared-prefix tensor-core tiles, split-KV worker "
+                              "with the store folded in, combine" if shared else
+                              "decode step: plan, split-KV worker with the store folded in, combine"),
                       achieved=attn_gbs, peak=peaks["hbm_gbs"], unit="GB/s",
                       frac=attn_gbs / peaks["hbm_gbs"], traffic=traffic,
                       peak_source=peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, burst copy)"),
@@ -520,6 +535,8 @@ def main(argv=None) -> int:
     ap.add_argument("--impl", choices=["nvpa", "reference"], default="nvpa")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--decode-api", choices=["shared", "plain"], default="shared",
+                    help="shared: nvpa_decode_step_shared_prefix; plain: nvpa_decode_step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -204,6 +204,55 @@ nvpa_status_t nvpa_decode_step(void* out, float* lse_out, const void* q,
                                cudaStream_t stream);
 
 /*
+ * Workspace for nvpa_decode_step_shared_prefix, in bytes, for the same arguments
+ * (host-side values only; 0 for invalid arguments).
+ */
+size_t nvpa_decode_shared_prefix_workspace_size(int batch, int num_q_heads, int num_kv_heads,
+                                                int head_dim, int max_context_len,
+                                                int block_size, int num_splits,
+                                                int min_group_size);
+
+/*
+ * nvpa_decode_step_shared_prefix -- the decode step of nvpa_decode_step (or, with
+ * k_new = v_new = slot_mapping = NULL, the attention of nvpa_paged_decode_attention) for
+ * batches in which many sequences share a cached prefix.  [P1] 4.2: prefix caching hands
+ * the blocks of an already cached prompt to every sequence that starts with it, raising
+ * the blocks' refcount, so those sequences' block tables begin with the same physical
+ * block ids.  The result is the same attention as nvpa_paged_decode_attention (up to
+ * floating-point rounding); only the schedule differs:
+ *  - sequences whose block_tables[b, 0] agree form a bucket; a bucket of at least
+ *    min_group_size sequences is a group.  The group's prefix is the longest run of
+ *    leading blocks that all members' tables hold, counting only blocks that lie
+ *    wholly before each member's newest key (position context_lens[b] - 1);
+ *  - each group's prefix keys are attended once for all its members on the tensor
+ *    cores (every member's query rows against the same K/V tiles), in partitions;
+ *  - the worker reads only each member's remaining keys; the combine merges the
+ *    prefix and private partitions with their log-sum-exp weights.
+ * Sequences in no group are decoded exactly as by nvpa_decode_step.  A batch above
+ * 2048 sequences is decoded without groups.  The fused store writes only position
+ * context_lens[b] - 1, which is never inside a group's prefix.
+ *
+ *   k_new, v_new,   as for nvpa_decode_step, or all three NULL (no store).
+ *   slot_mapping
+ *   min_group_size  smallest group (0 = the library default, 8; values below 2 act as 2).
+ *   workspace       at least nvpa_decode_shared_prefix_workspace_size(...) bytes,
+ *                   256-byte aligned.  After the call its first 256 bytes hold int32
+ *                   counters the plan wrote: [2] groups found, [3] sequences in them,
+ *                   [4] prefix tile entries (diagnostics; read after the stream syncs).
+ *   other arguments as for nvpa_decode_step.
+ * Errors: as nvpa_decode_step; a mix of NULL and non-NULL k_new/v_new/slot_mapping is
+ * NVPA_ERR_INVALID_ARG.
+ */
+nvpa_status_t nvpa_decode_step_shared_prefix(
+    void* out, float* lse_out, const void* q, const void* k_new, const void* v_new,
+    int64_t k_token_stride, int64_t v_token_stride, void* k_cache, void* v_cache,
+    const int32_t* slot_mapping, const int32_t* block_tables, int max_blocks_per_seq,
+    const int32_t* context_lens, int batch, int num_q_heads, int num_kv_heads, int head_dim,
+    int num_blocks, int block_size, int max_context_len, float softmax_scale, int num_splits,
+    int min_group_size, void* workspace, size_t workspace_bytes, int32_t* err_flag,
+    cudaStream_t stream);
+
+/*
  * nvpa_paged_decode_attention_static_scratch -- the same decode attention for callers
  * that cannot allocate device memory: a plugin inside a host runtime whose memory
  * manager owns all device memory and offers no allocation hook, or code running where an

@@ -15,7 +15,9 @@ from ._lib import (  # noqa: F401
     lib,
 )
 from .api import (  # noqa: F401
+    decode_shared_prefix_workspace_size,
     decode_step,
+    decode_step_shared_prefix,
     gather_kv,
     paged_decode_attention,
     paged_decode_workspace_size,

@@ -39,6 +39,10 @@ SIGNATURES = {
                                          _i, _f, _i, _p, _sz, _p, _p]),
     "nvpa_decode_step": (_i, [_p, _p, _p, _p, _p, _i64, _i64, _p, _p, _p, _p, _i, _p, _i, _i, _i,
                               _i, _i, _i, _i, _f, _i, _p, _sz, _p, _p]),
+    "nvpa_decode_shared_prefix_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i]),
+    "nvpa_decode_step_shared_prefix": (_i, [_p, _p, _p, _p, _p, _i64, _i64, _p, _p, _p, _p, _i, _p,
+                                            _i, _i, _i, _i, _i, _i, _i, _f, _i, _i, _p, _sz, _p,
+                                            _p]),
     "nvpa_paged_decode_attention_static_scratch": (_i, [_p, _p, _p, _p, _p, _p, _i, _p, _i, _i,
                                                         _i, _i, _i, _i, _i, _f, _i, _p, _p]),
     "nvpa_varlen_prefill_workspace_size": (_sz, [_i, _i]),

@@ -150,6 +150,60 @@ def decode_step(q, k_new, v_new, k_cache, v_cache, slot_mapping, block_tables, c
     return (out, lse) if return_lse else out
 
 
+def decode_shared_prefix_workspace_size(batch, num_q_heads, num_kv_heads, head_dim,
+                                        max_context_len, block_size, num_splits=0,
+                                        min_group_size=0) -> int:
+    return int(lib().nvpa_decode_shared_prefix_workspace_size(
+        batch, num_q_heads, num_kv_heads, head_dim, max_context_len, block_size, num_splits,
+        min_group_size))
+
+
+def decode_step_shared_prefix(q, k_new, v_new, k_cache, v_cache, slot_mapping, block_tables,
+                              context_lens, max_context_len, softmax_scale, out=None, lse=None,
+                              workspace=None, num_splits=0, min_group_size=0, err_flag=None,
+                              stream=None, return_lse=False):
+    """decode_step (or, with k_new = v_new = slot_mapping = None, paged_decode_attention)
+    with each group of sequences that share leading cache blocks attending its shared
+    prefix once, on the tensor cores."""
+    nb, bs, hkv, d = _cache_dims(k_cache, v_cache)
+    _need(q, _BF16, "q", 3)
+    _contig(q, "q")
+    b, hq, dq = (int(x) for x in q.shape)
+    if dq != d:
+        raise ValueError("q head_dim differs from the cache's")
+    store = k_new is not None
+    if store != (v_new is not None) or store != (slot_mapping is not None):
+        raise ValueError("k_new, v_new and slot_mapping must be given together")
+    if store:
+        for name, t in (("k_new", k_new), ("v_new", v_new)):
+            _need(t, _BF16, name, 3)
+            if tuple(t.shape) != (b, hkv, d) or t.stride(2) != 1 or t.stride(1) != d:
+                raise ValueError(f"{name} must be [{b}, {hkv}, {d}] with contiguous heads and dims")
+        _need(slot_mapping, _I32, "slot_mapping")
+        _contig(slot_mapping, "slot_mapping")
+    for name, t in (("block_tables", block_tables), ("context_lens", context_lens)):
+        _need(t, _I32, name)
+        _contig(t, name)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((b, hq), dtype=torch.float32, device=q.device)
+    need = decode_shared_prefix_workspace_size(b, hq, hkv, d, max_context_len, bs, num_splits,
+                                               min_group_size)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = lib().nvpa_decode_step_shared_prefix(
+        _ptr(out), _ptr(lse), _ptr(q), _ptr(k_new), _ptr(v_new),
+        k_new.stride(0) if store else 0, v_new.stride(0) if store else 0,
+        _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), _ptr(block_tables),
+        int(block_tables.shape[1]), _ptr(context_lens), b, hq, hkv, d, nb, bs,
+        int(max_context_len), float(softmax_scale), int(num_splits), int(min_group_size),
+        _ptr(workspace), int(workspace.numel() * workspace.element_size()), _ptr(err_flag),
+        _stream_handle(stream))
+    check(st, "nvpa_decode_step_shared_prefix")
+    return (out, lse) if return_lse else out
+
+
 def varlen_prefill_workspace_size(batch, total_q) -> int:
     return int(lib().nvpa_varlen_prefill_workspace_size(batch, total_q))
 

@@ -165,6 +165,58 @@ nvpa_status_t nvpa_paged_decode_attention(void* out, float* lse_out, const void*
     return run_paged_decode(c, stream);
 }
 
+static nvpa_status_t decode_step_common(void* out, float* lse_out, const void* q, const void* k_new,
+                                        const void* v_new, int64_t k_token_stride, int64_t v_token_stride,
+                                        void* k_cache, void* v_cache, const int32_t* slot_mapping,
+                                        const int32_t* block_tables, int max_blocks_per_seq,
+                                        const int32_t* context_lens, int batch, int num_q_heads,
+                                        int num_kv_heads, int head_dim, int num_blocks, int block_size,
+                                        int max_context_len, float softmax_scale, int num_splits,
+                                        bool store_optional, int shared_prefix, int min_group,
+                                        void* workspace, size_t workspace_bytes, int32_t* err_flag,
+                                        cudaStream_t stream) {
+    g_last_error[0] = 0;
+    NVPA_REQUIRE(batch >= 0 && max_context_len >= 0 && num_splits >= 0 && min_group >= 0,
+                 NVPA_ERR_INVALID_ARG, "batch, max_context_len, num_splits and min_group_size must be >= 0");
+    nvpa_status_t st = check_attention_shapes(num_q_heads, num_kv_heads, head_dim, num_blocks,
+                                              block_size, max_blocks_per_seq);
+    if (st != NVPA_OK) return st;
+    NVPA_REQUIRE(std::isfinite(softmax_scale), NVPA_ERR_INVALID_ARG, "softmax_scale not finite");
+    if (batch == 0) return NVPA_OK;
+    const bool any_new = k_new || v_new || slot_mapping;
+    const bool all_new = k_new && v_new && slot_mapping;
+    NVPA_REQUIRE(all_new || (store_optional && !any_new), NVPA_ERR_INVALID_ARG,
+                 store_optional ? "k_new, v_new and slot_mapping must be all set or all null"
+                                : "null pointer");
+    NVPA_REQUIRE(out && q && k_cache && v_cache && block_tables && context_lens && workspace,
+                 NVPA_ERR_INVALID_ARG, "null pointer");
+    if (all_new) {
+        const int64_t row = (int64_t)num_kv_heads * head_dim;
+        NVPA_REQUIRE(k_token_stride >= row && v_token_stride >= row && k_token_stride % 8 == 0 &&
+                         v_token_stride % 8 == 0,
+                     NVPA_ERR_INVALID_ARG, "token strides must be >= num_kv_heads*head_dim and multiples of 8");
+        NVPA_REQUIRE(aligned16(k_new) && aligned16(v_new), NVPA_ERR_INVALID_ARG,
+                     "bf16 pointers must be 16-byte aligned");
+    }
+    NVPA_REQUIRE(aligned16(out) && aligned16(q) && aligned16(k_cache) && aligned16(v_cache),
+                 NVPA_ERR_INVALID_ARG, "bf16 pointers must be 16-byte aligned");
+    NVPA_REQUIRE((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0, NVPA_ERR_INVALID_ARG,
+                 "workspace must be 256-byte aligned");
+    DecodeCall c{out, lse_out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                 batch, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, max_context_len,
+                 softmax_scale, num_splits, workspace, workspace_bytes, err_flag};
+    if (all_new) {
+        c.k_new = k_new;
+        c.v_new = v_new;
+        c.k_new_stride = k_token_stride;
+        c.v_new_stride = v_token_stride;
+        c.slot_mapping = slot_mapping;
+    }
+    c.shared_prefix = shared_prefix;
+    c.min_group = min_group;
+    return run_paged_decode(c, stream);
+}
+
 nvpa_status_t nvpa_decode_step(void* out, float* lse_out, const void* q, const void* k_new,
                                const void* v_new, int64_t k_token_stride, int64_t v_token_stride,
                                void* k_cache, void* v_cache, const int32_t* slot_mapping,
@@ -174,35 +226,37 @@ nvpa_status_t nvpa_decode_step(void* out, float* lse_out, const void* q, const v
                                int max_context_len, float softmax_scale, int num_splits,
                                void* workspace, size_t workspace_bytes, int32_t* err_flag,
                                cudaStream_t stream) {
-    g_last_error[0] = 0;
-    NVPA_REQUIRE(batch >= 0 && max_context_len >= 0 && num_splits >= 0, NVPA_ERR_INVALID_ARG,
-                 "batch, max_context_len and num_splits must be >= 0");
-    nvpa_status_t st = check_attention_shapes(num_q_heads, num_kv_heads, head_dim, num_blocks,
-                                              block_size, max_blocks_per_seq);
-    if (st != NVPA_OK) return st;
-    NVPA_REQUIRE(std::isfinite(softmax_scale), NVPA_ERR_INVALID_ARG, "softmax_scale not finite");
-    if (batch == 0) return NVPA_OK;
-    NVPA_REQUIRE(out && q && k_new && v_new && k_cache && v_cache && slot_mapping && block_tables &&
-                     context_lens && workspace,
-                 NVPA_ERR_INVALID_ARG, "null pointer");
-    const int64_t row = (int64_t)num_kv_heads * head_dim;
-    NVPA_REQUIRE(k_token_stride >= row && v_token_stride >= row && k_token_stride % 8 == 0 &&
-                     v_token_stride % 8 == 0,
-                 NVPA_ERR_INVALID_ARG, "token strides must be >= num_kv_heads*head_dim and multiples of 8");
-    NVPA_REQUIRE(aligned16(out) && aligned16(q) && aligned16(k_cache) && aligned16(v_cache) &&
-                     aligned16(k_new) && aligned16(v_new),
-                 NVPA_ERR_INVALID_ARG, "bf16 pointers must be 16-byte aligned");
-    NVPA_REQUIRE((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0, NVPA_ERR_INVALID_ARG,
-                 "workspace must be 256-byte aligned");
-    DecodeCall c{out, lse_out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
-                 batch, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, max_context_len,
-                 softmax_scale, num_splits, workspace, workspace_bytes, err_flag};
-    c.k_new = k_new;
-    c.v_new = v_new;
-    c.k_new_stride = k_token_stride;
-    c.v_new_stride = v_token_stride;
-    c.slot_mapping = slot_mapping;
-    return run_paged_decode(c, stream);
+    return decode_step_common(out, lse_out, q, k_new, v_new, k_token_stride, v_token_stride, k_cache,
+                              v_cache, slot_mapping, block_tables, max_blocks_per_seq, context_lens,
+                              batch, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size,
+                              max_context_len, softmax_scale, num_splits, false, 0, 0, workspace,
+                              workspace_bytes, err_flag, stream);
+}
+
+size_t nvpa_decode_shared_prefix_workspace_size(int batch, int num_q_heads, int num_kv_heads,
+                                                int head_dim, int max_context_len, int block_size,
+                                                int num_splits, int min_group_size) {
+    (void)block_size;
+    if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_context_len < 0 ||
+        num_splits < 0 || min_group_size < 0 || num_q_heads % num_kv_heads != 0)
+        return 0;
+    return decode_shared_prefix_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim,
+                                                max_context_len, num_splits, min_group_size);
+}
+
+nvpa_status_t nvpa_decode_step_shared_prefix(
+    void* out, float* lse_out, const void* q, const void* k_new, const void* v_new,
+    int64_t k_token_stride, int64_t v_token_stride, void* k_cache, void* v_cache,
+    const int32_t* slot_mapping, const int32_t* block_tables, int max_blocks_per_seq,
+    const int32_t* context_lens, int batch, int num_q_heads, int num_kv_heads, int head_dim,
+    int num_blocks, int block_size, int max_context_len, float softmax_scale, int num_splits,
+    int min_group_size, void* workspace, size_t workspace_bytes, int32_t* err_flag,
+    cudaStream_t stream) {
+    return decode_step_common(out, lse_out, q, k_new, v_new, k_token_stride, v_token_stride, k_cache,
+                              v_cache, slot_mapping, block_tables, max_blocks_per_seq, context_lens,
+                              batch, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size,
+                              max_context_len, softmax_scale, num_splits, true, 1, min_group_size,
+                              workspace, workspace_bytes, err_flag, stream);
 }
 
 size_t nvpa_varlen_prefill_workspace_size(int batch, int total_q) {

@@ -36,6 +36,10 @@ struct DecodeCall {
     const void* v_new = nullptr;
     long long k_new_stride = 0, v_new_stride = 0;
     const int32_t* slot_mapping = nullptr;
+    // shared-prefix decode (nvpa_decode_step_shared_prefix): group sequences whose block
+    // tables start with the same blocks and attend each group's prefix once
+    int shared_prefix = 0;
+    int min_group = 0;
 };
 
 struct PrefillCall {
@@ -55,9 +59,38 @@ struct PrefillCall {
     int32_t* err_flag;
 };
 
+// Shared-prefix part of a decode: every group's members (query rows) against the group's
+// prefix keys on the tensor cores; partition c of a prefix lands in slot c of each member's
+// split-KV partials.  The tables come from the decode plan (the kernel waits for it).
+struct DecodePrefixArgs {
+    const void* q;
+    const void* k_cache;
+    const void* v_cache;
+    const int32_t* block_tables;
+    int max_blocks_per_seq;
+    int batch, hq, hkv, head_dim, num_blocks, block_size;
+    float scale;
+    int32_t* err_flag;
+    const int2* tiles;           // (group, query tile | partition << 16)
+    const int32_t* ntiles;
+    const int32_t* members;
+    const int32_t* group_start;
+    const int32_t* group_len;
+    float* o_part;
+    float* lse_part;
+    int s_max, pchunk;
+    long long max_entries;       // host bound on the number of tile entries
+};
+// Query heads that share one 128-row tensor-core tile (the group size when it is a power
+// of two up to 8, else 1).
+int attention_tile_pack(int hq, int hkv);
+cudaError_t launch_decode_prefix_tcgen05(const DecodePrefixArgs& a, cudaStream_t stream);
+
 int decode_chunk_keys(int batch, int num_kv_heads, int max_context_len, int num_splits);
 size_t decode_workspace_bytes(int batch, int hq, int hkv, int head_dim, int max_context_len,
                               int num_splits);
+size_t decode_shared_prefix_workspace_bytes(int batch, int hq, int hkv, int head_dim,
+                                            int max_context_len, int num_splits, int min_group);
 nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream);
 size_t prefill_workspace_bytes(int batch, int total_q);
 nvpa_status_t run_varlen_prefill_tcgen05(const PrefillCall& c, void* workspace, size_t workspace_bytes,

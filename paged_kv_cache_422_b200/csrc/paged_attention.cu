@@ -20,6 +20,7 @@
 // and query head) merges them with the log-sum-exp weights:
 //     lse = log sum_p exp(lse_p),   out = sum_p exp(lse_p - lse) * o_p.
 #include <algorithm>
+#include <climits>
 #include <mutex>
 
 #include "attn_warp.cuh"
@@ -33,6 +34,8 @@ namespace nvpa {
 
 constexpr int kAttnWarps = 4;
 constexpr int kAttnStages = NVPA_DECODE_STAGES;
+constexpr int kSharedMaxBatch = 2048;   // larger batches are decoded without prefix groups
+constexpr int kDefaultMinGroup = 8;
 
 struct AttnParams {
     const uint16_t* q;
@@ -63,6 +66,12 @@ struct AttnParams {
     int max_ctx;                   // host-side bound of context_lens
     int chunk, s_max;              // keys per partition, partitions of the longest context
     float scale_log2;
+    // shared-prefix plan outputs (decode_plan_shared_kernel)
+    int2* ptiles;                  // (group, query tile | prefix partition << 16)
+    int32_t* members;              // grouped member lists
+    int32_t* group_start;          // [groups + 1]
+    int32_t* group_len;            // [groups] prefix tokens
+    int min_members, pchunk, ptq;  // smallest group, prefix keys per partition, members per tile
 };
 
 template <int D, int GMAX>
@@ -132,6 +141,198 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const AttnParams p) {
     if (tid == 0) {
         p.counter[0] = 0;
         p.counter[1] = carry_s * p.hkv;
+        p.counter[2] = p.counter[3] = p.counter[4] = 0;   // no shared-prefix groups
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// shared-prefix plan
+// ------------------------------------------------------------------------------------
+// Prefix caching hands a cached prompt's blocks to every sequence that starts with it, by
+// reference count ("Nano-vLLM part 1" section 4.2), so such sequences' block tables begin
+// with the same physical block ids.  This plan buckets the sequences by their first block
+// id (open addressing in shared memory); a bucket with at least min_members sequences is a
+// group, and the group's prefix is the longest run of leading blocks that every member
+// holds, counting only blocks that lie wholly before each member's newest token (that
+// token is written in this step).  Each member's context then splits into
+//   prefix partitions  0 .. npc-1       keys [c * pchunk, ...) of the prefix, computed once
+//                                        for all members on the tensor cores;
+//   private partitions npc .. npc+nsp-1 keys [prefix + s * chunk, ...), worker items;
+// and the combine merges all npc + nsp partials.  Sequences outside a group get the plain
+// decode plan's items.  Counters in the workspace: [0] next item, [1] items, [2] groups,
+// [3] members, [4] prefix tile entries.
+constexpr int kSharedTable = 2 * kSharedMaxBatch;   // a power of two above the batch
+
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& total) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    if (lane == 31) warp_tot[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+        int w = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += n;
+        }
+        warp_tot[lane] = w;
+    }
+    __syncthreads();
+    const int excl = incl - v + (wid ? warp_tot[wid - 1] : 0);
+    total = warp_tot[31];
+    __syncthreads();
+    return excl;
+}
+
+__global__ void __launch_bounds__(1024) decode_plan_shared_kernel(const AttnParams p) {
+    extern __shared__ int sh[];
+    int* tkey = sh;                            // first block id of the bucket, -1 = empty
+    int* tlead = tkey + kSharedTable;          // smallest member; later the member fill count
+    int* tcnt = tlead + kSharedTable;          // sequences in the bucket
+    int* tpref = tcnt + kSharedTable;          // prefix blocks: min over the members
+    int* tgid = tpref + kSharedTable;          // group id, -1 = not a group
+    int* tmst = tgid + kSharedTable;           // first index of the group in members[]
+    int* s_slot = tmst + kSharedTable;         // bucket of each sequence; later its prefix tokens
+    int* s_ctx = s_slot + kSharedMaxBatch;     // clamped context length
+    __shared__ int warp_tot[32];
+    __shared__ int s_ntiles;
+    const int tid = threadIdx.x;
+    pdl_launch_dependents();
+    for (int i = tid; i < kSharedTable; i += blockDim.x) {
+        tkey[i] = -1;
+        tlead[i] = INT_MAX;
+        tcnt[i] = 0;
+        tpref[i] = INT_MAX;
+        tgid[i] = -1;
+    }
+    if (tid == 0) s_ntiles = 0;
+    __syncthreads();
+    const int lim = (int)min((long long)p.max_ctx, (long long)p.max_blocks * p.block_size);
+
+    // 1. bucket by first block
+    for (int b = tid; b < p.batch; b += blockDim.x) {
+        int ctx = __ldg(p.context_lens + b);
+        if (ctx < 0 || ctx > lim) {
+            flag_error(p.err, NVPA_FLAG_BAD_LENGTH);
+            ctx = min(max(ctx, 0), lim);
+        }
+        s_ctx[b] = ctx;
+        int slot = -1;
+        const int full = ctx > 0 ? (ctx - 1) >> p.block_shift : 0;   // blocks before the newest token
+        if (full >= 1) {
+            const int key = __ldg(p.block_tables + (size_t)b * p.max_blocks);
+            if (key >= 0 && key < p.num_blocks) {
+                int h = (int)(((uint32_t)key * 2654435761u) >> 20) & (kSharedTable - 1);
+                while (true) {   // at most batch < kSharedTable buckets are taken
+                    const int prev = atomicCAS(tkey + h, -1, key);
+                    if (prev == -1 || prev == key) break;
+                    h = (h + 1) & (kSharedTable - 1);
+                }
+                slot = h;
+                atomicMin(tlead + h, b);
+                atomicAdd(tcnt + h, 1);
+            }
+        }
+        s_slot[b] = slot;
+    }
+    __syncthreads();
+
+    // 2. prefix of each bucket that is large enough: common leading blocks with its
+    //    smallest member, at most the blocks before each member's newest token
+    for (int b = tid; b < p.batch; b += blockDim.x) {
+        const int slot = s_slot[b];
+        if (slot < 0 || tcnt[slot] < p.min_members) continue;
+        const int full = (s_ctx[b] - 1) >> p.block_shift;
+        const int32_t* bb = p.block_tables + (size_t)b * p.max_blocks;
+        const int32_t* bl = p.block_tables + (size_t)tlead[slot] * p.max_blocks;
+        int n = 1;   // block 0 is the bucket key
+        while (n < full && __ldg(bb + n) == __ldg(bl + n)) ++n;
+        atomicMin(tpref + slot, n);
+    }
+    __syncthreads();
+
+    // 3. number the groups (in bucket order), place their member lists, list their tiles
+    constexpr int PER = kSharedTable / 1024;
+    bool used[PER];
+    int v = 0;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const int i = tid * PER + u;
+        used[u] = i < kSharedTable && tkey[i] >= 0 && tcnt[i] >= p.min_members && tpref[i] != INT_MAX;
+        if (used[u]) v += (tcnt[i] << 12) + 1;   // members in the high bits, groups in the low 12
+    }
+    int tot = 0;
+    int excl = block_exclusive_scan(v, warp_tot, tot);
+    int g = excl & 4095, m = excl >> 12;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        if (!used[u]) continue;
+        const int i = tid * PER + u;
+        const int cnt = tcnt[i];
+        const int pre = tpref[i] << p.block_shift;
+        tgid[i] = g;
+        tmst[i] = m;
+        tlead[i] = 0;
+        p.group_start[g] = m;
+        p.group_len[g] = pre;
+        const int nq = (cnt + p.ptq - 1) / p.ptq;
+        const int nch = (pre + p.pchunk - 1) / p.pchunk;
+        const int off = atomicAdd(&s_ntiles, nq * nch);
+        for (int c = 0; c < nch; ++c)
+            for (int qt = 0; qt < nq; ++qt) p.ptiles[off + c * nq + qt] = make_int2(g, qt | (c << 16));
+        ++g;
+        m += cnt;
+    }
+    const int ngroups = tot & 4095, nmembers = tot >> 12;
+    if (tid == 0) p.group_start[ngroups] = nmembers;
+    __syncthreads();
+
+    // 4. members and partition counts
+    for (int b = tid; b < p.batch; b += blockDim.x) {
+        const int slot = s_slot[b];
+        const int gid = slot >= 0 ? tgid[slot] : -1;
+        int pre = 0;
+        if (gid >= 0) {
+            const int pos = atomicAdd(tlead + slot, 1);
+            p.members[tmst[slot] + pos] = b;
+            pre = tpref[slot] << p.block_shift;
+        }
+        const int npc = (pre + p.pchunk - 1) / p.pchunk;
+        const int nsp = max(1, (s_ctx[b] - pre + p.chunk - 1) / p.chunk);
+        p.nsplit[b] = npc + nsp;
+        s_slot[b] = pre;
+    }
+    __syncthreads();
+
+    // 5. worker items for the private partitions
+    int carry = 0;
+    for (int base = 0; base < p.batch; base += blockDim.x) {
+        const int b = base + tid;
+        int nsp = 0, npc = 0, pre = 0, ctx = 0;
+        if (b < p.batch) {
+            pre = s_slot[b];
+            ctx = s_ctx[b];
+            npc = (pre + p.pchunk - 1) / p.pchunk;
+            nsp = max(1, (ctx - pre + p.chunk - 1) / p.chunk);
+        }
+        int block_tot = 0;
+        const int e = carry + block_exclusive_scan(nsp, warp_tot, block_tot);
+        for (int s = 0; s < nsp; ++s)
+            p.items[e + s] = make_int4(b, (npc + s) | ((npc + nsp) << 16), pre + s * p.chunk,
+                                       min(ctx, pre + (s + 1) * p.chunk));
+        carry += block_tot;
+    }
+    if (tid == 0) {
+        p.counter[0] = 0;
+        p.counter[1] = carry * p.hkv;
+        p.counter[2] = ngroups;
+        p.counter[3] = nmembers;
+        p.counter[4] = s_ntiles;
     }
 }
 
@@ -483,10 +684,12 @@ cudaError_t dispatch_worker(const AttnParams& p, int head_dim, long long max_ite
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct DecodeWorkspace {
-    size_t counter, nsplit, items, lse_part, o_part, total;
+    size_t counter, nsplit, items, lse_part, o_part, members, group_start, group_len, ptiles, total;
 };
 
-DecodeWorkspace decode_workspace_layout(int batch, int hq, int hkv, int head_dim, int s_max) {
+// ptile_entries > 0: room for the shared-prefix plan's tables as well
+DecodeWorkspace decode_workspace_layout(int batch, int hq, int hkv, int head_dim, int s_max,
+                                        long long ptile_entries = 0) {
     (void)hkv;
     DecodeWorkspace w;
     size_t off = 0;
@@ -497,9 +700,43 @@ DecodeWorkspace decode_workspace_layout(int batch, int hq, int hkv, int head_dim
     off = align256(off + (s_max > 1 ? sizeof(float) * (size_t)batch * hq * s_max : 0));
     w.o_part = off;
     off = align256(off + (s_max > 1 ? sizeof(float) * (size_t)batch * hq * s_max * head_dim : 0));
+    w.members = w.group_start = w.group_len = w.ptiles = off;
+    if (ptile_entries > 0) {
+        w.members = off; off = align256(off + sizeof(int32_t) * (size_t)batch);
+        w.group_start = off; off = align256(off + sizeof(int32_t) * ((size_t)batch + 1));
+        w.group_len = off; off = align256(off + sizeof(int32_t) * (size_t)batch);
+        w.ptiles = off; off = align256(off + sizeof(int2) * (size_t)ptile_entries);
+    }
     w.total = off;
     return w;
 }
+
+// Partitioning of a shared-prefix decode; active == false when the batch is too large
+// for the plan's table (the call then runs as a plain decode step).
+struct SharedGeometry {
+    bool active;
+    int chunk, s_max, pchunk, ptq, min_members;
+    long long entries;   // bound on prefix tile entries
+};
+
+SharedGeometry shared_geometry(int batch, int hq, int hkv, int max_context_len, int num_splits,
+                               int min_group) {
+    SharedGeometry g{};
+    g.chunk = decode_chunk_keys(batch, hkv, max_context_len, num_splits);
+    const int ctx = std::max(0, max_context_len);
+    g.active = batch <= kSharedMaxBatch;
+    // one more partition than a plain decode: splitting a context at the prefix boundary
+    // adds at most one (pchunk >= chunk)
+    g.s_max = std::max(1, (ctx + g.chunk - 1) / g.chunk) + (g.active ? 1 : 0);
+    g.pchunk = (g.chunk + 127) / 128 * 128;
+    g.ptq = 128 / attention_tile_pack(hq, hkv);
+    g.min_members = min_group > 0 ? std::max(2, min_group) : kDefaultMinGroup;
+    const long long groups = batch / g.min_members;
+    g.entries = g.active ? ((long long)batch / g.ptq + groups + 1) * ((ctx + g.pchunk - 1) / g.pchunk + 1) : 0;
+    return g;
+}
+
+constexpr size_t kSharedPlanSmem = sizeof(int) * (6 * (size_t)kSharedTable + 2 * (size_t)kSharedMaxBatch);
 
 }  // namespace
 
@@ -522,10 +759,20 @@ size_t decode_workspace_bytes(int batch, int hq, int hkv, int head_dim, int max_
     return decode_workspace_layout(batch, hq, hkv, head_dim, s_max).total;
 }
 
+size_t decode_shared_prefix_workspace_bytes(int batch, int hq, int hkv, int head_dim,
+                                            int max_context_len, int num_splits, int min_group) {
+    const SharedGeometry g = shared_geometry(batch, hq, hkv, max_context_len, num_splits, min_group);
+    return decode_workspace_layout(batch, hq, hkv, head_dim, g.s_max, g.entries).total;
+}
+
 nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream) {
+    const SharedGeometry sg = c.shared_prefix
+        ? shared_geometry(c.batch, c.hq, c.hkv, c.max_context_len, c.num_splits, c.min_group)
+        : SharedGeometry{};
+    const bool shared = c.shared_prefix && sg.active;
     const int chunk = decode_chunk_keys(c.batch, c.hkv, c.max_context_len, c.num_splits);
-    const int s_max = std::max(1, (std::max(0, c.max_context_len) + chunk - 1) / chunk);
-    const DecodeWorkspace w = decode_workspace_layout(c.batch, c.hq, c.hkv, c.head_dim, s_max);
+    const int s_max = c.shared_prefix ? sg.s_max : std::max(1, (std::max(0, c.max_context_len) + chunk - 1) / chunk);
+    const DecodeWorkspace w = decode_workspace_layout(c.batch, c.hq, c.hkv, c.head_dim, s_max, sg.entries);
     if (c.workspace_bytes < w.total) {
         set_error("workspace too small: %zu bytes given, %zu needed", c.workspace_bytes, w.total);
         return NVPA_ERR_WORKSPACE_TOO_SMALL;
@@ -567,10 +814,59 @@ nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream) {
     p.k_cache_w = static_cast<uint16_t*>(const_cast<void*>(c.k_cache));
     p.v_cache_w = static_cast<uint16_t*>(const_cast<void*>(c.v_cache));
 
-    decode_plan_kernel<<<1, 1024, 0, stream>>>(p);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_failure(e, "decode plan launch");
-    count_launches(1);
+    cudaError_t e = cudaSuccess;
+    if (shared) {
+        p.ptiles = reinterpret_cast<int2*>(ws + w.ptiles);
+        p.members = reinterpret_cast<int32_t*>(ws + w.members);
+        p.group_start = reinterpret_cast<int32_t*>(ws + w.group_start);
+        p.group_len = reinterpret_cast<int32_t*>(ws + w.group_len);
+        p.min_members = sg.min_members;
+        p.pchunk = sg.pchunk;
+        p.ptq = sg.ptq;
+        static std::once_flag once[64];
+        int dev = 0;
+        cudaGetDevice(&dev);
+        std::call_once(once[dev & 63], [] {
+            cudaFuncSetAttribute(decode_plan_shared_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kSharedPlanSmem);
+        });
+        decode_plan_shared_kernel<<<1, 1024, kSharedPlanSmem, stream>>>(p);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_failure(e, "decode plan launch");
+        count_launches(1);
+        DecodePrefixArgs a{};
+        a.q = c.q;
+        a.k_cache = c.k_cache;
+        a.v_cache = c.v_cache;
+        a.block_tables = c.block_tables;
+        a.max_blocks_per_seq = c.max_blocks_per_seq;
+        a.batch = c.batch;
+        a.hq = c.hq;
+        a.hkv = c.hkv;
+        a.head_dim = c.head_dim;
+        a.num_blocks = c.num_blocks;
+        a.block_size = c.block_size;
+        a.scale = c.scale;
+        a.err_flag = c.err_flag;
+        a.tiles = p.ptiles;
+        a.ntiles = p.counter + 4;
+        a.members = p.members;
+        a.group_start = p.group_start;
+        a.group_len = p.group_len;
+        a.o_part = p.o_part;
+        a.lse_part = p.lse_part;
+        a.s_max = s_max;
+        a.pchunk = sg.pchunk;
+        a.max_entries = sg.entries;
+        e = launch_decode_prefix_tcgen05(a, stream);
+        if (e != cudaSuccess) return cuda_failure(e, "decode shared-prefix launch");
+        count_launches(1);
+    } else {
+        decode_plan_kernel<<<1, 1024, 0, stream>>>(p);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_failure(e, "decode plan launch");
+        count_launches(1);
+    }
     const long long max_items = (long long)c.batch * c.hkv * s_max;
     e = dispatch_worker(p, c.head_dim, max_items, stream);
     if (e != cudaSuccess) return cuda_failure(e, "decode worker launch");

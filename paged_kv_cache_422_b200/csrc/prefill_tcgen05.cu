@@ -64,6 +64,16 @@ struct PrefillParams {
     int32_t* err;
     const int2* tiles;           // plan: (sequence, query tile), longest first
     const int32_t* ntiles;       // plan: number of entries
+    // shared-prefix decode mode: "sequences" are prefix groups whose "queries" are the
+    // members' decode query rows; results go to each member's prefix partition slot
+    const uint16_t* q_rows;      // decode q [batch, Hq, D]
+    const int32_t* members;      // members of all groups, grouped
+    const int32_t* group_start;  // [num_groups + 1] into members
+    const int32_t* group_len;    // [num_groups] shared prefix length in tokens
+    float* o_part;               // partition c of the prefix goes to slot c of each member
+    float* lse_part;
+    int s_max;
+    int pchunk;                  // prefix keys per partition (a multiple of 128)
     int batch, total_q, hq, hkv, group;
     int pack, pack_shift;        // query heads per row group (P) and log2(P)
     int tq;                      // tokens per tile, 128 / P
@@ -94,6 +104,7 @@ struct Layout {
 struct TileInfo {
     int seq, qt, head0, hk;
     int q0, lq, lk;      // first query row (global), query rows, keys of the sequence
+    int kbeg, chunk;     // shared-prefix mode: first key and index of the key partition
     int tok0, ntok;      // first token of the tile inside the sequence, tokens in the tile
     int nkv;             // key tiles visited
 };
@@ -103,19 +114,32 @@ __device__ __forceinline__ int tile_nkv(int causal, int lq, int lk, int tok0, in
     return causal ? min(ktiles, (lk - lq + tok0 + ntok - 1) / kKV + 1) : ktiles;
 }
 
+template <bool PREFIX>
 __device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, int idx) {
     TileInfo t;
     const int2 e = __ldg(p.tiles + idx / p.hgroups);
     t.seq = e.x;
-    t.qt = e.y;
+    t.qt = e.y & 0xffff;
     t.head0 = (idx % p.hgroups) * p.pack;
     t.hk = t.head0 / p.group;
-    t.q0 = __ldg(p.cu_q + t.seq);
-    t.lq = __ldg(p.cu_q + t.seq + 1) - t.q0;
-    t.lk = __ldg(p.cu_k + t.seq + 1) - __ldg(p.cu_k + t.seq);
+    if constexpr (PREFIX) {
+        // group e.x: its members are the queries, keys [kbeg, kbeg + lk) of its shared
+        // prefix the keys (no mask)
+        t.chunk = e.y >> 16;
+        t.kbeg = t.chunk * p.pchunk;
+        t.q0 = __ldg(p.group_start + t.seq);
+        t.lq = __ldg(p.group_start + t.seq + 1) - t.q0;
+        t.lk = min(p.pchunk, __ldg(p.group_len + t.seq) - t.kbeg);
+    } else {
+        t.chunk = 0;
+        t.kbeg = 0;
+        t.q0 = __ldg(p.cu_q + t.seq);
+        t.lq = __ldg(p.cu_q + t.seq + 1) - t.q0;
+        t.lk = __ldg(p.cu_k + t.seq + 1) - __ldg(p.cu_k + t.seq);
+    }
     t.tok0 = t.qt * p.tq;
     t.ntok = min(p.tq, t.lq - t.tok0);
-    t.nkv = tile_nkv(p.causal, t.lq, t.lk, t.tok0, t.ntok);
+    t.nkv = tile_nkv(PREFIX ? 0 : p.causal, t.lq, t.lk, t.tok0, t.ntok);
     return t;
 }
 
@@ -245,7 +269,7 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const PrefillParams 
 // ------------------------------------------------------------------------------------
 // the attention kernel
 // ------------------------------------------------------------------------------------
-template <int D>
+template <int D, bool PREFIX>
 __global__ void __launch_bounds__(kThreads, 2)
 prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap k_map,
                        const __grid_constant__ CUtensorMap v_map, const PrefillParams p) {
@@ -260,6 +284,12 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if constexpr (PREFIX) {
+        // shared-prefix mode follows the decode plan: let the worker's CTAs launch as this
+        // grid's CTAs finish, and wait for the plan's tables
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+    }
 
     if (threadIdx.x == 0) {
         mbar_init(bars + L::B_QFULL, 1);
@@ -302,12 +332,12 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
         int last_fill[kStages];
         for (int s = 0; s < kStages; ++s) last_fill[s] = -1;
         const int piece = min(p.block_size, kKV);
-        auto load_pieces = [&](const int32_t* bt, int lk, int j) {
+        auto load_pieces = [&](const int32_t* bt, int kbeg, int lk, int j) {
             const int key0 = j * kKV;
             const int npieces = (min(kKV, lk - key0) + piece - 1) / piece;
             int blk = -1;
             if (lane < npieces) {
-                blk = __ldg(bt + ((key0 + lane * piece) >> p.block_shift));
+                blk = __ldg(bt + ((kbeg + key0 + lane * piece) >> p.block_shift));
                 if (blk < 0 || blk >= p.num_blocks) {
                     flag_error(p.err, NVPA_FLAG_BAD_BLOCK_ID);
                     blk = -1;
@@ -316,19 +346,42 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             return blk;
         };
         for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
-            const TileInfo t = tile_info(p, idx);
-            const int32_t* bt = p.block_tables + (size_t)t.seq * p.max_blocks;
-            int cur_blk = load_pieces(bt, t.lk, 0);
+            const TileInfo t = tile_info<PREFIX>(p, idx);
+            const int bt_seq = PREFIX ? __ldg(p.members + t.q0) : t.seq;   // a member's table
+            const int32_t* bt = p.block_tables + (size_t)bt_seq * p.max_blocks;
+            int cur_blk = load_pieces(bt, t.kbeg, t.lk, 0);
             if (!mbar_wait(bars + L::B_QEMPTY, (tcount & 1) ^ 1, abort_flag, p.err)) break;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(bars + L::B_QFULL, L::TILE_BYTES);
-                for (int r = 0; r < L::REGIONS; ++r)
-                    tma_load_3d(smem + L::Q_OFF + r * L::REGION_BYTES, &q_map, bars + L::B_QFULL, r * 64,
-                                t.head0, t.q0 + t.tok0);
+            if constexpr (PREFIX) {
+                // gather the members' query rows into the swizzled Q tile: row r is member
+                // tok0 + r / P, head head0 + r % P; 16-byte chunk c of a 128-byte row goes to
+                // chunk c ^ (r % 8) (the 128-byte swizzle the MMA descriptors expect)
+                for (int e = lane; e < kQ * (D / 8); e += 32) {
+                    const int r = e / (D / 8), c = e % (D / 8);
+                    const int mi = t.tok0 + (r >> p.pack_shift);
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (mi < t.lq) {
+                        const int b = __ldg(p.members + t.q0 + mi);
+                        const uint16_t* src = p.q_rows + ((size_t)b * p.hq + t.head0 + (r & (p.pack - 1))) * D + c * 8;
+                        v = __ldg(reinterpret_cast<const uint4*>(src));
+                    }
+                    const int region = c / 8, cc = c % 8;
+                    *reinterpret_cast<uint4*>(smem + L::Q_OFF + region * L::REGION_BYTES + r * 128 +
+                                              ((cc ^ (r & 7)) * 16)) = v;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars + L::B_QFULL);
+            } else {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bars + L::B_QFULL, L::TILE_BYTES);
+                    for (int r = 0; r < L::REGIONS; ++r)
+                        tma_load_3d(smem + L::Q_OFF + r * L::REGION_BYTES, &q_map, bars + L::B_QFULL, r * 64,
+                                    t.head0, t.q0 + t.tok0);
+                }
             }
             bool ok = true;
             for (int j = 0; j < t.nkv && ok; ++j) {
-                const int nxt_blk = j + 1 < t.nkv ? load_pieces(bt, t.lk, j + 1) : -1;
+                const int nxt_blk = j + 1 < t.nkv ? load_pieces(bt, t.kbeg, t.lk, j + 1) : -1;
                 const int key0 = j * kKV;
                 const uint32_t valid_mask = __ballot_sync(0xffffffffu, cur_blk >= 0);
                 const uint32_t bytes = (uint32_t)__popc(valid_mask) * (uint32_t)(piece * 128 * L::REGIONS);
@@ -345,7 +398,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                         const int c = __ffs(m) - 1;
                         const int blk = __shfl_sync(0xffffffffu, cur_blk, c);
                         if (lane == 0) {
-                            const int kc = key0 + c * piece;
+                            const int kc = t.kbeg + key0 + c * piece;
                             const int z = blk * p.block_size + (kc & (p.block_size - 1));
                             for (int r = 0; r < L::REGIONS; ++r)
                                 tma_load_3d(dst + r * L::REGION_BYTES + c * piece * 128, map,
@@ -385,7 +438,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
         uint32_t p_use = 0;
         bool ok = true;
         for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
-            const TileInfo t = tile_info(p, idx);
+            const TileInfo t = tile_info<PREFIX>(p, idx);
             if (!mbar_wait(bars + L::B_QFULL, tcount & 1, abort_flag, p.err)) break;
             for (int j = 0; j < t.nkv && ok; ++j) {
                 // S_j = Q K_j^T
@@ -476,9 +529,9 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
         int tcount = 0;
         uint32_t pv_before = 0;                       // PVs issued for earlier tiles
         for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
-            const TileInfo t = tile_info(p, idx);
+            const TileInfo t = tile_info<PREFIX>(p, idx);
             const int pos = t.lk - t.lq + t.tok0 + rtok;           // absolute position of this row
-            const int lim = p.causal ? min(t.lk, pos + 1) : t.lk;  // keys 0 .. lim-1 are visible
+            const int lim = (!PREFIX && p.causal) ? min(t.lk, pos + 1) : t.lk;  // keys 0 .. lim-1 visible
             const int lim_min = __reduce_min_sync(0xffffffffu, lim);
             float m = -INFINITY, l = 0.f;
             bool ok = true;
@@ -491,77 +544,81 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                 tc_fence_after();
                 const int key0 = j * kKV;
                 const bool open = key0 + kKV <= lim_min;          // no mask anywhere in the warp
-                // P_j against the current reference max, packed bf16 pairs in registers
-                uint32_t pk[kKV / 2];
-                float mt = -INFINITY, lt = 0.f;
-                const float m_use = m == -INFINITY ? INFINITY : m;   // first tile: all weights 0 for now
+                // the whole S_j row in registers: four loads, one wait
+                uint32_t sv[kKV];
 #pragma unroll
-                for (int c = 0; c < kKV / 32; ++c) {
-                    uint32_t sv[32];
-                    tmem_ld32(s_col + c * 32, sv);
-                    tmem_wait_ld();
+                for (int c = 0; c < kKV / 32; ++c)
+                    tmem_ld32(s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
+                tmem_wait_ld();
+                // pass 1: row max of the visible raw scores (min too, for a negative scale)
+                float hi = -INFINITY, lo = INFINITY;
+                if (open) {
 #pragma unroll
-                    for (int k = 0; k < 32; k += 2) {
-                        float x0 = __uint_as_float(sv[k]) * p.scale_log2;
-                        float x1 = __uint_as_float(sv[k + 1]) * p.scale_log2;
-                        if (!open) {
-                            x0 = (key0 + c * 32 + k < lim) ? x0 : -INFINITY;
-                            x1 = (key0 + c * 32 + k + 1 < lim) ? x1 : -INFINITY;
-                        }
-                        mt = fmaxf(mt, fmaxf(x0, x1));
-                        const float a = fast_exp2(x0 - m_use), b = fast_exp2(x1 - m_use);
-                        lt += a + b;
-                        pk[c * 16 + k / 2] = pack_bf16x2(a, b);
+                    for (int k = 0; k < kKV; ++k) {
+                        const float x = __uint_as_float(sv[k]);
+                        hi = fmaxf(hi, x);
+                        lo = fminf(lo, x);
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < kKV; ++k) {
+                        const float x = __uint_as_float(sv[k]);
+                        const bool vis = key0 + k < lim;
+                        hi = fmaxf(hi, vis ? x : -INFINITY);
+                        lo = fminf(lo, vis ? x : INFINITY);
                     }
                 }
+                const float sc = p.scale_log2;
+                const float mt = hi == -INFINITY ? -INFINITY : (sc >= 0.f ? hi * sc : lo * sc);
                 const bool over = mt > m + kRescaleSlack;
-                if (__any_sync(0xffffffffu, over)) {
+                const bool rescale = __any_sync(0xffffffffu, over);
+                float alpha = 1.f;
+                if (rescale) {
                     const float m_new = over ? mt : m;
-                    const float alpha = over ? (m == -INFINITY ? 0.f : fast_exp2(m - m_new)) : 1.f;
-                    if (j > 0) {
-                        // O holds P_0..P_{j-1} V: wait for the last of them, then rescale
-                        if (!mbar_wait(bars + L::B_ODONE, (pv_before + j - 1) & 1, abort_flag, p.err)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-#pragma unroll
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t o[32];
-                            tmem_ld32(o_col + c * 32, o);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-                            tmem_st32(o_col + c * 32, o);
-                        }
-                        tmem_wait_st();
-                    }
+                    alpha = over ? (m == -INFINITY ? 0.f : fast_exp2(m - m_new)) : 1.f;
                     l *= alpha;
                     m = m_new;
-                    // recompute P_j against the new reference (S_j is still intact)
-                    const bool live = m > -INFINITY;
-                    lt = 0.f;
+                }
+                // pass 2: P_j = exp2(s * scale - m) as bf16 pairs over the first kKV/2 columns of
+                // S_j; masked keys get 0 by select
+                const bool live = m > -INFINITY;
+                const float nm = -m;
 #pragma unroll
-                    for (int c = 0; c < kKV / 32; ++c) {
-                        uint32_t sv[32];
-                        tmem_ld32(s_col + c * 32, sv);
+                for (int c = 0; c < kKV / 32; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int k = 0; k < 32; k += 2) {
+                        const int kk = c * 32 + k;
+                        float a = fast_exp2(fmaf(__uint_as_float(sv[kk]), sc, nm));
+                        float b = fast_exp2(fmaf(__uint_as_float(sv[kk + 1]), sc, nm));
+                        if (!open) {
+                            a = (key0 + kk < lim) ? a : 0.f;
+                            b = (key0 + kk + 1 < lim) ? b : 0.f;
+                        }
+                        if (!live) a = b = 0.f;
+                        l += a + b;
+                        pk[k / 2] = pack_bf16x2(a, b);
+                    }
+                    tmem_st16(s_col + c * 16, pk);
+                }
+                if (rescale && j > 0) {
+                    // O holds P_0..P_{j-1} V (all complete once S_j is): rescale it before
+                    // P_j is released to the MMA
+                    if (!mbar_wait(bars + L::B_ODONE, (pv_before + j - 1) & 1, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(o_col + c * 32, o);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int k = 0; k < 32; k += 2) {
-                            float x0 = __uint_as_float(sv[k]) * p.scale_log2;
-                            float x1 = __uint_as_float(sv[k + 1]) * p.scale_log2;
-                            x0 = (key0 + c * 32 + k < lim) ? x0 : -INFINITY;
-                            x1 = (key0 + c * 32 + k + 1 < lim) ? x1 : -INFINITY;
-                            const float a = live ? fast_exp2(x0 - m) : 0.f;
-                            const float b = live ? fast_exp2(x1 - m) : 0.f;
-                            lt += a + b;
-                            pk[c * 16 + k / 2] = pack_bf16x2(a, b);
-                        }
+                        for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                        tmem_st32(o_col + c * 32, o);
                     }
                 }
-                l += lt;
-                tmem_st32(s_col, *reinterpret_cast<uint32_t(*)[32]>(pk));
-                tmem_st32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -572,8 +629,16 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             tc_fence_after();
             const bool row_ok = rtok < t.ntok;
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            const size_t orow = (size_t)(t.q0 + t.tok0 + rtok) * p.hq + t.head0 + rhead;
-            uint4* dst = reinterpret_cast<uint4*>(p.out + orow * D);
+            size_t orow;
+            float* pdst = nullptr;
+            if constexpr (PREFIX) {
+                const int b = row_ok ? __ldg(p.members + t.q0 + t.tok0 + rtok) : 0;
+                orow = ((size_t)b * p.hq + t.head0 + rhead) * p.s_max + t.chunk;
+                pdst = p.o_part + orow * D;
+            } else {
+                orow = (size_t)(t.q0 + t.tok0 + rtok) * p.hq + t.head0 + rhead;
+            }
+            uint4* dst = reinterpret_cast<uint4*>(p.out + (PREFIX ? 0 : orow * D));
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
@@ -584,7 +649,13 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bars + L::B_OFREE);
                 }
-                if (row_ok) {
+                if (PREFIX && row_ok) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        __stcg(reinterpret_cast<float4*>(pdst + c * 32 + 4 * q),
+                               make_float4(__uint_as_float(o[4 * q + 0]) * inv, __uint_as_float(o[4 * q + 1]) * inv,
+                                           __uint_as_float(o[4 * q + 2]) * inv, __uint_as_float(o[4 * q + 3]) * inv));
+                } else if (row_ok) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         uint4 w;
@@ -596,7 +667,11 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                     }
                 }
             }
-            if (row_ok && p.lse_out != nullptr) p.lse_out[orow] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+            if constexpr (PREFIX) {
+                if (row_ok) __stcg(p.lse_part + orow, l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY);
+            } else {
+                if (row_ok && p.lse_out != nullptr) p.lse_out[orow] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+            }
             pv_before += (uint32_t)t.nkv;
             ++tcount;
         }
@@ -645,21 +720,82 @@ bool make_map(CUtensorMap* map, const void* base, int dim, int heads, long long 
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, bool PREFIX>
 cudaError_t launch_prefill(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
                            const PrefillParams& p, int grid, cudaStream_t stream) {
     static std::once_flag once[64];
     int dev = 0;
     cudaGetDevice(&dev);
     std::call_once(once[dev & 63], [] {
-        cudaFuncSetAttribute(prefill_tcgen05_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(prefill_tcgen05_kernel<D, PREFIX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Layout<D>::ALLOC);
     });
-    prefill_tcgen05_kernel<D><<<grid, kThreads, Layout<D>::ALLOC, stream>>>(qm, km, vm, p);
-    return cudaGetLastError();
+    if constexpr (!PREFIX) {
+        prefill_tcgen05_kernel<D, false><<<grid, kThreads, Layout<D>::ALLOC, stream>>>(qm, km, vm, p);
+        return cudaGetLastError();
+    } else {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = Layout<D>::ALLOC;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, prefill_tcgen05_kernel<D, true>, qm, km, vm, p);
+    }
 }
 
 }  // namespace
+
+int attention_tile_pack(int hq, int hkv) {
+    const int group = hq / hkv;
+    return (group & (group - 1)) == 0 ? std::min(group, kQ / kMinTokensPerTile) : 1;
+}
+
+cudaError_t launch_decode_prefix_tcgen05(const DecodePrefixArgs& a, cudaStream_t stream) {
+    const int pack = attention_tile_pack(a.hq, a.hkv);
+    CUtensorMap km, vm;
+    const int box_kv = std::min(a.block_size, kKV);
+    if (!make_map(&km, a.k_cache, a.head_dim, a.hkv, (long long)a.num_blocks * a.block_size, 1, box_kv) ||
+        !make_map(&vm, a.v_cache, a.head_dim, a.hkv, (long long)a.num_blocks * a.block_size, 1, box_kv)) {
+        set_error("cuTensorMapEncodeTiled failed (driver entry point missing or bad layout)");
+        return cudaErrorInvalidValue;
+    }
+    PrefillParams p{};
+    p.block_tables = a.block_tables;
+    p.err = a.err_flag;
+    p.tiles = a.tiles;
+    p.ntiles = a.ntiles;
+    p.q_rows = static_cast<const uint16_t*>(a.q);
+    p.members = a.members;
+    p.group_start = a.group_start;
+    p.group_len = a.group_len;
+    p.o_part = a.o_part;
+    p.lse_part = a.lse_part;
+    p.s_max = a.s_max;
+    p.pchunk = a.pchunk;
+    p.batch = a.batch;
+    p.hq = a.hq;
+    p.hkv = a.hkv;
+    p.group = a.hq / a.hkv;
+    p.pack = pack;
+    p.pack_shift = __builtin_ctz((unsigned)pack);
+    p.tq = kQ / pack;
+    p.hgroups = a.hq / pack;
+    p.max_blocks = a.max_blocks_per_seq;
+    p.num_blocks = a.num_blocks;
+    p.block_size = a.block_size;
+    p.block_shift = __builtin_ctz((unsigned)a.block_size);
+    p.scale_log2 = a.scale * kLog2e;
+    const long long units = std::max(1LL, a.max_entries) * p.hgroups;
+    const int grid = (int)std::min<long long>(2LL * device_sm_count(), units);
+    // the query map is not read in this mode (rows are gathered); any valid map will do
+    return a.head_dim == 128 ? launch_prefill<128, true>(km, km, vm, p, grid, stream)
+                             : launch_prefill<64, true>(km, km, vm, p, grid, stream);
+}
 
 size_t prefill_workspace_bytes(int batch, int total_q) {
     const size_t entries = (size_t)std::max(0, batch) +
@@ -676,7 +812,7 @@ nvpa_status_t run_varlen_prefill_tcgen05(const PrefillCall& c, void* workspace, 
     }
     // query heads packed per 128-row tile: the group size when it is a power of two <= 8
     const int group = c.hq / c.hkv;
-    const int pack = (group & (group - 1)) == 0 ? std::min(group, kQ / kMinTokensPerTile) : 1;
+    const int pack = attention_tile_pack(c.hq, c.hkv);
     CUtensorMap qm, km, vm;
     const int box_kv = std::min(c.block_size, kKV);
     if (!make_map(&qm, c.q, c.head_dim, c.hq, c.total_q, pack, kQ / pack) ||
@@ -719,8 +855,8 @@ nvpa_status_t run_varlen_prefill_tcgen05(const PrefillCall& c, void* workspace, 
     count_launches(1);
     const long long max_tiles = ((long long)c.batch + (c.total_q + p.tq - 1) / p.tq) * p.hgroups;
     const int grid = (int)std::max(1LL, std::min<long long>(2LL * device_sm_count(), max_tiles));
-    e = c.head_dim == 128 ? launch_prefill<128>(qm, km, vm, p, grid, stream)
-                          : launch_prefill<64>(qm, km, vm, p, grid, stream);
+    e = c.head_dim == 128 ? launch_prefill<128, false>(qm, km, vm, p, grid, stream)
+                          : launch_prefill<64, false>(qm, km, vm, p, grid, stream);
     if (e != cudaSuccess) return cuda_failure(e, "prefill tcgen05 launch");
     count_launches(1);
     return NVPA_OK;
