@@ -284,6 +284,47 @@ nvpa_status_t nvpa_paged_decode_attention_static_scratch(
     int32_t* err_flag, cudaStream_t stream);
 
 /*
+ * nvpa_paged_decode_partial -- the decode attention of nvpa_paged_decode_attention over the
+ * keys this call sees, returned as a partial (fp32 output and log-sum-exp) for a later
+ * log-sum-exp merge: for long contexts whose keys are spread over several devices, each device runs
+ * this over its own key range (its own block tables and context lengths) and
+ * nvpa_lse_combine merges the parts (the split-KV combine of [P1] 5.2 decode, across
+ * devices; the exchange of the parts between devices is the caller's collective).
+ *
+ *   o_part          float32 [batch, num_q_heads, head_dim] (written): this call's output
+ *                   normalised over its own keys; all zeros for a sequence with no keys.
+ *   lse_part        float32 [batch, num_q_heads] (written): natural-log sum-exp of the
+ *                   scaled scores over this call's keys, -inf with no keys.  Required.
+ *   other arguments and the workspace as for nvpa_paged_decode_attention.
+ */
+nvpa_status_t nvpa_paged_decode_partial(float* o_part, float* lse_part, const void* q,
+                                        const void* k_cache, const void* v_cache,
+                                        const int32_t* block_tables, int max_blocks_per_seq,
+                                        const int32_t* context_lens, int batch, int num_q_heads,
+                                        int num_kv_heads, int head_dim, int num_blocks,
+                                        int block_size, int max_context_len, float softmax_scale,
+                                        int num_splits, void* workspace, size_t workspace_bytes,
+                                        int32_t* err_flag, cudaStream_t stream);
+
+/*
+ * nvpa_lse_combine -- merge num_parts partials of the same queries over disjoint key sets:
+ *     lse = log sum_r exp(lse_r),   out = sum_r exp(lse_r - lse) * o_r.
+ * A part with lse_r = -inf weighs 0; a row whose parts are all -inf gets out = 0 and
+ * lse = -inf.  The result equals attention over the union of the parts' keys up to
+ * floating-point rounding.
+ *
+ *   out             bf16 [batch, num_q_heads, head_dim] (written).
+ *   lse_out         float32 [batch, num_q_heads] (written) or NULL.
+ *   o_parts         float32 [num_parts, batch, num_q_heads, head_dim], 16-byte aligned.
+ *   lse_parts       float32 [num_parts, batch, num_q_heads].
+ *   head_dim        64 or 128.
+ * Errors: NVPA_ERR_INVALID_ARG (null, num_parts < 1, misaligned), NVPA_ERR_UNSUPPORTED.
+ */
+nvpa_status_t nvpa_lse_combine(void* out, float* lse_out, const float* o_parts,
+                               const float* lse_parts, int num_parts, int batch, int num_q_heads,
+                               int head_dim, cudaStream_t stream);
+
+/*
  * Workspace for nvpa_varlen_prefill_attention, in bytes (the query-tile schedule), for a
  * call with `batch` sequences and `total_q` query rows.  Host-side values only.
  */

@@ -19,7 +19,9 @@ from .api import (  # noqa: F401
     decode_step,
     decode_step_shared_prefix,
     gather_kv,
+    lse_combine,
     paged_decode_attention,
+    paged_decode_partial,
     paged_decode_workspace_size,
     store_kvcache,
     varlen_prefill_attention,

@@ -9,7 +9,10 @@ from __future__ import annotations
 import ctypes
 import os
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvpa.so")
+# NVPA_LIB names another build of the same library (a variant built with
+# `python -m paged_kv_cache_422_b200.build --out PATH`).
+LIB_PATH = os.environ.get("NVPA_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                                                       "libnvpa.so")
 
 NVPA_OK = 0
 NVPA_ERR_INVALID_ARG = 1
@@ -45,6 +48,9 @@ SIGNATURES = {
                                             _p]),
     "nvpa_paged_decode_attention_static_scratch": (_i, [_p, _p, _p, _p, _p, _p, _i, _p, _i, _i,
                                                         _i, _i, _i, _i, _i, _f, _i, _p, _p]),
+    "nvpa_paged_decode_partial": (_i, [_p, _p, _p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i,
+                                       _f, _i, _p, _sz, _p, _p]),
+    "nvpa_lse_combine": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _p]),
     "nvpa_varlen_prefill_workspace_size": (_sz, [_i, _i]),
     "nvpa_varlen_prefill_attention": (_i, [_p, _p, _p, _p, _p, _p, _i, _p, _p, _i, _i, _i, _i,
                                            _i, _i, _i, _i, _i, _f, _i, _p, _sz, _p, _p]),

@@ -257,3 +257,55 @@ def gather_kv(cache, block_tables, cu_seqlens_k, total_k, out=None, err_flag=Non
                               _ptr(err_flag), _stream_handle(stream))
     check(st, "nvpa_gather_kv")
     return out
+
+
+def paged_decode_partial(q, k_cache, v_cache, block_tables, context_lens, max_context_len,
+                         softmax_scale, o_part=None, lse_part=None, workspace=None, num_splits=0,
+                         err_flag=None, stream=None):
+    """Decode attention over the keys this call sees, as a partial for lse_combine:
+    (o_part [B, Hq, D] fp32 normalised over these keys, lse_part [B, Hq] fp32)."""
+    nb, bs, hkv, d = _cache_dims(k_cache, v_cache)
+    _need(q, _BF16, "q", 3)
+    _contig(q, "q")
+    b, hq, dq = (int(x) for x in q.shape)
+    if dq != d:
+        raise ValueError("q head_dim differs from the cache's")
+    for name, t in (("block_tables", block_tables), ("context_lens", context_lens)):
+        _need(t, _I32, name)
+        _contig(t, name)
+    if o_part is None:
+        o_part = torch.empty((b, hq, d), dtype=torch.float32, device=q.device)
+    if lse_part is None:
+        lse_part = torch.empty((b, hq), dtype=torch.float32, device=q.device)
+    _need(o_part, torch.float32, "o_part", 3)
+    _need(lse_part, torch.float32, "lse_part", 2)
+    need = paged_decode_workspace_size(b, hq, hkv, d, max_context_len, bs, num_splits)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = lib().nvpa_paged_decode_partial(
+        _ptr(o_part), _ptr(lse_part), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        int(block_tables.shape[1]), _ptr(context_lens), b, hq, hkv, d, nb, bs,
+        int(max_context_len), float(softmax_scale), int(num_splits), _ptr(workspace),
+        int(workspace.numel() * workspace.element_size()), _ptr(err_flag), _stream_handle(stream))
+    check(st, "nvpa_paged_decode_partial")
+    return o_part, lse_part
+
+
+def lse_combine(o_parts, lse_parts, out=None, lse_out=None, stream=None, return_lse=False):
+    """Merge partials over disjoint key sets: o_parts [R, B, Hq, D] fp32 and lse_parts
+    [R, B, Hq] fp32 -> out [B, Hq, D] bf16 (and lse [B, Hq])."""
+    _need(o_parts, torch.float32, "o_parts", 4)
+    _need(lse_parts, torch.float32, "lse_parts", 3)
+    _contig(o_parts, "o_parts")
+    _contig(lse_parts, "lse_parts")
+    r, b, hq, d = (int(x) for x in o_parts.shape)
+    if tuple(lse_parts.shape) != (r, b, hq):
+        raise ValueError(f"lse_parts must be [{r}, {b}, {hq}]")
+    if out is None:
+        out = torch.empty((b, hq, d), dtype=_BF16, device=o_parts.device)
+    if return_lse and lse_out is None:
+        lse_out = torch.empty((b, hq), dtype=torch.float32, device=o_parts.device)
+    st = lib().nvpa_lse_combine(_ptr(out), _ptr(lse_out), _ptr(o_parts), _ptr(lse_parts), r, b, hq,
+                                d, _stream_handle(stream))
+    check(st, "nvpa_lse_combine")
+    return (out, lse_out) if return_lse else out

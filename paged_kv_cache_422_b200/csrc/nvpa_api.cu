@@ -259,6 +259,53 @@ nvpa_status_t nvpa_decode_step_shared_prefix(
                               workspace, workspace_bytes, err_flag, stream);
 }
 
+nvpa_status_t nvpa_paged_decode_partial(float* o_part, float* lse_part, const void* q,
+                                        const void* k_cache, const void* v_cache,
+                                        const int32_t* block_tables, int max_blocks_per_seq,
+                                        const int32_t* context_lens, int batch, int num_q_heads,
+                                        int num_kv_heads, int head_dim, int num_blocks,
+                                        int block_size, int max_context_len, float softmax_scale,
+                                        int num_splits, void* workspace, size_t workspace_bytes,
+                                        int32_t* err_flag, cudaStream_t stream) {
+    g_last_error[0] = 0;
+    NVPA_REQUIRE(batch >= 0 && max_context_len >= 0 && num_splits >= 0, NVPA_ERR_INVALID_ARG,
+                 "batch, max_context_len and num_splits must be >= 0");
+    nvpa_status_t st = check_attention_shapes(num_q_heads, num_kv_heads, head_dim, num_blocks,
+                                              block_size, max_blocks_per_seq);
+    if (st != NVPA_OK) return st;
+    NVPA_REQUIRE(std::isfinite(softmax_scale), NVPA_ERR_INVALID_ARG, "softmax_scale not finite");
+    if (batch == 0) return NVPA_OK;
+    NVPA_REQUIRE(o_part && lse_part && q && k_cache && v_cache && block_tables && context_lens && workspace,
+                 NVPA_ERR_INVALID_ARG, "null pointer");
+    NVPA_REQUIRE(aligned16(o_part) && aligned16(q) && aligned16(k_cache) && aligned16(v_cache),
+                 NVPA_ERR_INVALID_ARG, "o_part and bf16 pointers must be 16-byte aligned");
+    NVPA_REQUIRE((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0, NVPA_ERR_INVALID_ARG,
+                 "workspace must be 256-byte aligned");
+    DecodeCall c{o_part, lse_part, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                 batch, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, max_context_len,
+                 softmax_scale, num_splits, workspace, workspace_bytes, err_flag};
+    c.out_f32 = o_part;
+    return run_paged_decode(c, stream);
+}
+
+nvpa_status_t nvpa_lse_combine(void* out, float* lse_out, const float* o_parts,
+                               const float* lse_parts, int num_parts, int batch, int num_q_heads,
+                               int head_dim, cudaStream_t stream) {
+    g_last_error[0] = 0;
+    NVPA_REQUIRE(num_parts >= 1 && batch >= 0 && num_q_heads > 0, NVPA_ERR_INVALID_ARG,
+                 "num_parts must be >= 1, batch >= 0 and num_q_heads > 0");
+    NVPA_REQUIRE(head_dim == 64 || head_dim == 128, NVPA_ERR_UNSUPPORTED,
+                 "head_dim %d not supported (64, 128)", head_dim);
+    NVPA_REQUIRE((long long)num_parts * batch * num_q_heads <= 0x7fffffffLL, NVPA_ERR_UNSUPPORTED,
+                 "num_parts * batch * num_q_heads above 2^31-1");
+    if (batch == 0) return NVPA_OK;
+    NVPA_REQUIRE(out && o_parts && lse_parts, NVPA_ERR_INVALID_ARG, "null pointer");
+    NVPA_REQUIRE(aligned16(out) && aligned16(o_parts), NVPA_ERR_INVALID_ARG,
+                 "out and o_parts must be 16-byte aligned");
+    return run_lse_combine(out, lse_out, o_parts, lse_parts, num_parts, batch, num_q_heads, head_dim,
+                           stream);
+}
+
 size_t nvpa_varlen_prefill_workspace_size(int batch, int total_q) {
     if (batch < 0 || total_q < 0) return 0;
     return prefill_workspace_bytes(batch, total_q);

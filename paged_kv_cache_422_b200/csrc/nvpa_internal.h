@@ -40,6 +40,8 @@ struct DecodeCall {
     // tables start with the same blocks and attend each group's prefix once
     int shared_prefix = 0;
     int min_group = 0;
+    // partial decode (nvpa_paged_decode_partial): fp32 normalised output here, `out` unused
+    float* out_f32 = nullptr;
 };
 
 struct PrefillCall {
@@ -80,6 +82,8 @@ struct DecodePrefixArgs {
     float* lse_part;
     int s_max, pchunk;
     long long max_entries;       // host bound on the number of tile entries
+    int max_ctas;                // grid cap (0: two per SM)
+    bool pdl;                    // launch as a programmatic dependent of the previous kernel
 };
 // Query heads that share one 128-row tensor-core tile (the group size when it is a power
 // of two up to 8, else 1).
@@ -95,6 +99,9 @@ nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream);
 size_t prefill_workspace_bytes(int batch, int total_q);
 nvpa_status_t run_varlen_prefill_tcgen05(const PrefillCall& c, void* workspace, size_t workspace_bytes,
                                          cudaStream_t stream);
+
+nvpa_status_t run_lse_combine(void* out, float* lse_out, const float* o_parts, const float* lse_parts,
+                              int num_parts, int batch, int hq, int head_dim, cudaStream_t stream);
 
 nvpa_status_t run_store_kvcache(const void* k, const void* v, int64_t k_stride, int64_t v_stride,
                                 void* k_cache, void* v_cache, const int32_t* slot_mapping,

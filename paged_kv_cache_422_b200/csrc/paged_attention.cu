@@ -54,6 +54,7 @@ struct AttnParams {
     uint16_t* k_cache_w;
     uint16_t* v_cache_w;
     uint16_t* out;
+    float* out_f32;                // partial mode: fp32 normalised output instead of bf16 `out`
     float* lse_out;
     float* o_part;
     float* lse_part;
@@ -217,6 +218,7 @@ __global__ void __launch_bounds__(1024) decode_plan_shared_kernel(const AttnPara
     // 1. bucket by first block
     for (int b = tid; b < p.batch; b += blockDim.x) {
         int ctx = __ldg(p.context_lens + b);
+        const int key = __ldg(p.block_tables + (size_t)b * p.max_blocks);   // loaded alongside
         if (ctx < 0 || ctx > lim) {
             flag_error(p.err, NVPA_FLAG_BAD_LENGTH);
             ctx = min(max(ctx, 0), lim);
@@ -225,7 +227,6 @@ __global__ void __launch_bounds__(1024) decode_plan_shared_kernel(const AttnPara
         int slot = -1;
         const int full = ctx > 0 ? (ctx - 1) >> p.block_shift : 0;   // blocks before the newest token
         if (full >= 1) {
-            const int key = __ldg(p.block_tables + (size_t)b * p.max_blocks);
             if (key >= 0 && key < p.num_blocks) {
                 int h = (int)(((uint32_t)key * 2654435761u) >> 20) & (kSharedTable - 1);
                 while (true) {   // at most batch < kSharedTable buckets are taken
@@ -250,8 +251,24 @@ __global__ void __launch_bounds__(1024) decode_plan_shared_kernel(const AttnPara
         const int full = (s_ctx[b] - 1) >> p.block_shift;
         const int32_t* bb = p.block_tables + (size_t)b * p.max_blocks;
         const int32_t* bl = p.block_tables + (size_t)tlead[slot] * p.max_blocks;
-        int n = 1;   // block 0 is the bucket key
-        while (n < full && __ldg(bb + n) == __ldg(bl + n)) ++n;
+        // common leading blocks with the smallest member, compared 8 entries at a time
+        // (independent loads); block 0 is the bucket key
+        int n = 1;
+        bool run = true;
+        while (run && n < full) {
+            int eb[8], el[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const bool in = n + u < full;
+                eb[u] = in ? __ldg(bb + n + u) : 0;
+                el[u] = in ? __ldg(bl + n + u) : 1;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (run && eb[u] == el[u]) ++n;
+                else run = false;
+            }
+        }
         atomicMin(tpref + slot, n);
     }
     __syncthreads();
@@ -481,7 +498,12 @@ paged_attention_kernel(const AttnParams p) {
                 float v[8];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) acc.out_pair(g, k, v[2 * k], v[2 * k + 1]);
-                if (ns == 1) {
+                if (ns == 1 && p.out_f32 != nullptr) {
+                    float* op = p.out_f32 + ((size_t)qrow * p.hq + h) * D + sub * 8;
+                    *reinterpret_cast<float4*>(op) = make_float4(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv);
+                    *reinterpret_cast<float4*>(op + 4) = make_float4(v[4] * inv, v[5] * inv, v[6] * inv, v[7] * inv);
+                    if (sub == 0 && p.lse_out != nullptr) p.lse_out[(size_t)qrow * p.hq + h] = lse;
+                } else if (ns == 1) {
                     uint4 w;
                     w.x = pack_bf16x2(v[0] * inv, v[1] * inv);
                     w.y = pack_bf16x2(v[2] * inv, v[3] * inv);
@@ -604,6 +626,13 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const AttnParams p)
         tot = warp_sum(tot);
     }
     const float inv = tot > 0.f ? 1.f / tot : 0.f;
+    if (p.out_f32 != nullptr) {
+        float* dst = p.out_f32 + (size_t)w * D + lane * DPL;
+#pragma unroll
+        for (int k = 0; k < DPL; ++k) dst[k] = acc[k] * inv;
+        if (lane == 0 && p.lse_out != nullptr) p.lse_out[w] = tot > 0.f ? mx + __logf(tot) : -INFINITY;
+        return;
+    }
     uint16_t* dst = p.out + (size_t)w * D + lane * DPL;
     if constexpr (DPL == 4) {
         uint2 v;
@@ -682,6 +711,7 @@ cudaError_t dispatch_worker(const AttnParams& p, int head_dim, long long max_ite
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
 
 struct DecodeWorkspace {
     size_t counter, nsplit, items, lse_part, o_part, members, group_start, group_len, ptiles, total;
@@ -785,6 +815,7 @@ nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream) {
     p.block_tables = c.block_tables;
     p.context_lens = c.context_lens;
     p.out = static_cast<uint16_t*>(c.out);
+    p.out_f32 = c.out_f32;
     p.lse_out = c.lse_out;
     p.counter = reinterpret_cast<int32_t*>(ws + w.counter);
     p.nsplit = reinterpret_cast<int32_t*>(ws + w.nsplit);
@@ -858,6 +889,7 @@ nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream) {
         a.s_max = s_max;
         a.pchunk = sg.pchunk;
         a.max_entries = sg.entries;
+        a.pdl = true;
         e = launch_decode_prefix_tcgen05(a, stream);
         if (e != cudaSuccess) return cuda_failure(e, "decode shared-prefix launch");
         count_launches(1);

@@ -54,6 +54,91 @@ constexpr int kStages = 2;       // K/V ring stages, each one K or one V tile
 constexpr int kThreads = 192;    // 6 warps
 constexpr int kTmemCols = 256;   // S/P 128 + O up to 128
 constexpr int kMinTokensPerTile = 16;   // 128 rows / at most 8 packed heads
+// Bit k set for the first n of 32 columns (n clamped to [0, 32]).
+__device__ __forceinline__ uint32_t visible_mask(int n) {
+    return n >= 32 ? 0xffffffffu : n <= 0 ? 0u : ((1u << n) - 1u);
+}
+
+// bits as a float when bit k of vm is set, else `fill` (shift/and/or, no predicate).
+__device__ __forceinline__ float keep_or(uint32_t bits, uint32_t vm, int k, float fill) {
+    const uint32_t keep = (uint32_t)((int32_t)(vm << (31 - k)) >> 31);
+    return __uint_as_float((bits & keep) | (__float_as_uint(fill) & ~keep));
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+__device__ __forceinline__ float min3(float a, float b, float c) {
+    float d;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Max (MAX) or min of the visible raw scores of one 128-column S row; with MASK only the
+// columns below lim - key0 count (masked ones become -inf / +inf by bit mask).  Two
+// independent accumulators, two new scores per three-input instruction.
+template <bool MAX, bool MASK>
+__device__ __forceinline__ float row_extreme(const uint32_t (&sv)[kKV], int key0, int lim) {
+    const float fill = MAX ? -INFINITY : INFINITY;
+    float e0 = fill, e1 = fill;
+#pragma unroll
+    for (int c = 0; c < kKV / 32; ++c) {
+        const uint32_t vm = MASK ? visible_mask(lim - key0 - c * 32) : 0xffffffffu;
+#pragma unroll
+        for (int k = 0; k < 32; k += 4) {
+            float x0 = __uint_as_float(sv[c * 32 + k]), x1 = __uint_as_float(sv[c * 32 + k + 1]);
+            float x2 = __uint_as_float(sv[c * 32 + k + 2]), x3 = __uint_as_float(sv[c * 32 + k + 3]);
+            if (MASK) {
+                x0 = keep_or(sv[c * 32 + k], vm, k, fill);
+                x1 = keep_or(sv[c * 32 + k + 1], vm, k + 1, fill);
+                x2 = keep_or(sv[c * 32 + k + 2], vm, k + 2, fill);
+                x3 = keep_or(sv[c * 32 + k + 3], vm, k + 3, fill);
+            }
+            e0 = MAX ? max3(e0, x0, x1) : min3(e0, x0, x1);
+            e1 = MAX ? max3(e1, x2, x3) : min3(e1, x2, x3);
+        }
+    }
+    return MAX ? fmaxf(e0, e1) : fminf(e0, e1);
+}
+
+// P = exp2(s * sce + nme) of one S row, packed to bf16 pairs and written over the first
+// kKV/2 TMEM columns of the row (32 S columns become 16 P columns, each chunk's P landing
+// in columns already read); returns the row sum of the fp32 values.  With MASK, columns
+// at or past lim - key0 get 0 by bit mask.
+template <bool MASK>
+__device__ __forceinline__ float exp_row(const uint32_t (&sv)[kKV], uint32_t s_col, float sce, float nme,
+                                         int key0, int lim) {
+    float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+#pragma unroll
+    for (int c = 0; c < kKV / 32; ++c) {
+        const uint32_t vm = MASK ? visible_mask(lim - key0 - c * 32) : 0xffffffffu;
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 32; k += 4) {
+            float p0 = fast_exp2(fmaf(__uint_as_float(sv[c * 32 + k]), sce, nme));
+            float p1 = fast_exp2(fmaf(__uint_as_float(sv[c * 32 + k + 1]), sce, nme));
+            float p2 = fast_exp2(fmaf(__uint_as_float(sv[c * 32 + k + 2]), sce, nme));
+            float p3 = fast_exp2(fmaf(__uint_as_float(sv[c * 32 + k + 3]), sce, nme));
+            if (MASK) {
+                p0 = keep_or(__float_as_uint(p0), vm, k, 0.f);
+                p1 = keep_or(__float_as_uint(p1), vm, k + 1, 0.f);
+                p2 = keep_or(__float_as_uint(p2), vm, k + 2, 0.f);
+                p3 = keep_or(__float_as_uint(p3), vm, k + 3, 0.f);
+            }
+            l0 += p0;
+            l1 += p1;
+            l2 += p2;
+            l3 += p3;
+            pk[k / 2] = pack_bf16x2(p0, p1);
+            pk[k / 2 + 1] = pack_bf16x2(p2, p3);
+        }
+        tmem_st16(s_col + c * 16, pk);
+    }
+    return (l0 + l1) + (l2 + l3);
+}
 
 struct PrefillParams {
     const int32_t* block_tables;
@@ -352,22 +437,32 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             int cur_blk = load_pieces(bt, t.kbeg, t.lk, 0);
             if (!mbar_wait(bars + L::B_QEMPTY, (tcount & 1) ^ 1, abort_flag, p.err)) break;
             if constexpr (PREFIX) {
-                // gather the members' query rows into the swizzled Q tile: row r is member
-                // tok0 + r / P, head head0 + r % P; 16-byte chunk c of a 128-byte row goes to
-                // chunk c ^ (r % 8) (the 128-byte swizzle the MMA descriptors expect)
-                for (int e = lane; e < kQ * (D / 8); e += 32) {
-                    const int r = e / (D / 8), c = e % (D / 8);
+                // gather the members' query rows into the swizzled Q tile with 16-byte
+                // cp.async copies, all in flight at once: lane l fills rows l, l+32, l+64,
+                // l+96; row r is member tok0 + r / P, head head0 + r % P, and 16-byte chunk c
+                // of its 128-byte half goes to chunk c ^ (r % 8) (the 128-byte swizzle the
+                // MMA descriptors expect).  Rows past the group are zero-filled.
+                const uint16_t* src[kQ / 32];
+#pragma unroll
+                for (int i = 0; i < kQ / 32; ++i) {
+                    const int r = lane + 32 * i;
                     const int mi = t.tok0 + (r >> p.pack_shift);
-                    uint4 v = make_uint4(0, 0, 0, 0);
-                    if (mi < t.lq) {
-                        const int b = __ldg(p.members + t.q0 + mi);
-                        const uint16_t* src = p.q_rows + ((size_t)b * p.hq + t.head0 + (r & (p.pack - 1))) * D + c * 8;
-                        v = __ldg(reinterpret_cast<const uint4*>(src));
-                    }
-                    const int region = c / 8, cc = c % 8;
-                    *reinterpret_cast<uint4*>(smem + L::Q_OFF + region * L::REGION_BYTES + r * 128 +
-                                              ((cc ^ (r & 7)) * 16)) = v;
+                    const int b = mi < t.lq ? __ldg(p.members + t.q0 + mi) : -1;
+                    src[i] = b < 0 ? nullptr
+                                   : p.q_rows + ((size_t)b * p.hq + t.head0 + (r & (p.pack - 1))) * D;
                 }
+#pragma unroll
+                for (int i = 0; i < kQ / 32; ++i) {
+                    const int r = lane + 32 * i;
+#pragma unroll
+                    for (int c = 0; c < D / 8; ++c) {
+                        uint8_t* dst = smem + L::Q_OFF + (c / 8) * L::REGION_BYTES + r * 128 +
+                                       (((c % 8) ^ (r & 7)) * 16);
+                        cp_async16(dst, src[i] != nullptr ? src[i] + c * 8 : p.q_rows, src[i] != nullptr ? 16 : 0);
+                    }
+                }
+                cp_async_commit();
+                cp_async_wait<0>();
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bars + L::B_QFULL);
@@ -550,26 +645,17 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                 for (int c = 0; c < kKV / 32; ++c)
                     tmem_ld32(s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
                 tmem_wait_ld();
-                // pass 1: row max of the visible raw scores (min too, for a negative scale)
-                float hi = -INFINITY, lo = INFINITY;
-                if (open) {
-#pragma unroll
-                    for (int k = 0; k < kKV; ++k) {
-                        const float x = __uint_as_float(sv[k]);
-                        hi = fmaxf(hi, x);
-                        lo = fminf(lo, x);
-                    }
-                } else {
-#pragma unroll
-                    for (int k = 0; k < kKV; ++k) {
-                        const float x = __uint_as_float(sv[k]);
-                        const bool vis = key0 + k < lim;
-                        hi = fmaxf(hi, vis ? x : -INFINITY);
-                        lo = fminf(lo, vis ? x : INFINITY);
-                    }
-                }
+                // pass 1: the row's largest visible scaled score: the max of the raw scores
+                // for a positive scale, the min for a negative one.  The softmax is bound by
+                // the ALU pipe (min/max, selects, packing), so tiles that need no mask take a
+                // loop of three-input max/min and nothing else.
                 const float sc = p.scale_log2;
-                const float mt = hi == -INFINITY ? -INFINITY : (sc >= 0.f ? hi * sc : lo * sc);
+                float ext;
+                if (open)
+                    ext = sc >= 0.f ? row_extreme<true, false>(sv, key0, lim) : row_extreme<false, false>(sv, key0, lim);
+                else
+                    ext = sc >= 0.f ? row_extreme<true, true>(sv, key0, lim) : row_extreme<false, true>(sv, key0, lim);
+                const float mt = fabsf(ext) == INFINITY ? -INFINITY : ext * sc;
                 const bool over = mt > m + kRescaleSlack;
                 const bool rescale = __any_sync(0xffffffffu, over);
                 float alpha = 1.f;
@@ -579,28 +665,13 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                     l *= alpha;
                     m = m_new;
                 }
-                // pass 2: P_j = exp2(s * scale - m) as bf16 pairs over the first kKV/2 columns of
-                // S_j; masked keys get 0 by select
+                // pass 2: P_j = exp2(s * scale - m) as bf16 pairs over the first kKV/2 columns
+                // of S_j.  A row with no visible key yet (m = -inf) gets exp2(-inf) = 0
+                // through its operands, not through a select per element.
                 const bool live = m > -INFINITY;
-                const float nm = -m;
-#pragma unroll
-                for (int c = 0; c < kKV / 32; ++c) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int k = 0; k < 32; k += 2) {
-                        const int kk = c * 32 + k;
-                        float a = fast_exp2(fmaf(__uint_as_float(sv[kk]), sc, nm));
-                        float b = fast_exp2(fmaf(__uint_as_float(sv[kk + 1]), sc, nm));
-                        if (!open) {
-                            a = (key0 + kk < lim) ? a : 0.f;
-                            b = (key0 + kk + 1 < lim) ? b : 0.f;
-                        }
-                        if (!live) a = b = 0.f;
-                        l += a + b;
-                        pk[k / 2] = pack_bf16x2(a, b);
-                    }
-                    tmem_st16(s_col + c * 16, pk);
-                }
+                const float sce = live ? sc : 0.f, nme = live ? -m : -INFINITY;
+                l += open ? exp_row<false>(sv, s_col, sce, nme, key0, lim)
+                          : exp_row<true>(sv, s_col, sce, nme, key0, lim);
                 if (rescale && j > 0) {
                     // O holds P_0..P_{j-1} V (all complete once S_j is): rescale it before
                     // P_j is released to the MMA
@@ -722,7 +793,7 @@ bool make_map(CUtensorMap* map, const void* base, int dim, int heads, long long 
 
 template <int D, bool PREFIX>
 cudaError_t launch_prefill(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
-                           const PrefillParams& p, int grid, cudaStream_t stream) {
+                           const PrefillParams& p, int grid, cudaStream_t stream, bool pdl = PREFIX) {
     static std::once_flag once[64];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -730,8 +801,8 @@ cudaError_t launch_prefill(const CUtensorMap& qm, const CUtensorMap& km, const C
         cudaFuncSetAttribute(prefill_tcgen05_kernel<D, PREFIX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Layout<D>::ALLOC);
     });
-    if constexpr (!PREFIX) {
-        prefill_tcgen05_kernel<D, false><<<grid, kThreads, Layout<D>::ALLOC, stream>>>(qm, km, vm, p);
+    if (!pdl) {
+        prefill_tcgen05_kernel<D, PREFIX><<<grid, kThreads, Layout<D>::ALLOC, stream>>>(qm, km, vm, p);
         return cudaGetLastError();
     } else {
         cudaLaunchConfig_t cfg = {};
@@ -744,7 +815,7 @@ cudaError_t launch_prefill(const CUtensorMap& qm, const CUtensorMap& km, const C
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, prefill_tcgen05_kernel<D, true>, qm, km, vm, p);
+        return cudaLaunchKernelEx(&cfg, prefill_tcgen05_kernel<D, PREFIX>, qm, km, vm, p);
     }
 }
 
@@ -791,10 +862,11 @@ cudaError_t launch_decode_prefix_tcgen05(const DecodePrefixArgs& a, cudaStream_t
     p.block_shift = __builtin_ctz((unsigned)a.block_size);
     p.scale_log2 = a.scale * kLog2e;
     const long long units = std::max(1LL, a.max_entries) * p.hgroups;
-    const int grid = (int)std::min<long long>(2LL * device_sm_count(), units);
+    const long long cap = a.max_ctas > 0 ? a.max_ctas : 2LL * device_sm_count();
+    const int grid = (int)std::max(1LL, std::min<long long>(cap, units));
     // the query map is not read in this mode (rows are gathered); any valid map will do
-    return a.head_dim == 128 ? launch_prefill<128, true>(km, km, vm, p, grid, stream)
-                             : launch_prefill<64, true>(km, km, vm, p, grid, stream);
+    return a.head_dim == 128 ? launch_prefill<128, true>(km, km, vm, p, grid, stream, a.pdl)
+                             : launch_prefill<64, true>(km, km, vm, p, grid, stream, a.pdl);
 }
 
 size_t prefill_workspace_bytes(int batch, int total_q) {
