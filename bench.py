@@ -177,11 +177,10 @@ def profile_traffic(kernel_tag: str, source_files) -> float | None:
     return float(m.group(1))
 
 
+# sources of the split-KV worker, the dominant kernel of a decode step
 DECODE_SOURCES = ["paged_kv_cache_422_b200/csrc/paged_attention.cu",
                   "paged_kv_cache_422_b200/csrc/attn_warp.cuh",
-                  "paged_kv_cache_422_b200/csrc/common.cuh",
-                  "paged_kv_cache_422_b200/csrc/prefill_tcgen05.cu",
-                  "paged_kv_cache_422_b200/csrc/sm100.cuh"]
+                  "paged_kv_cache_422_b200/csrc/common.cuh"]
 
 
 def source_sha(files) -> str:
@@ -330,6 +329,12 @@ def run_nvpa(args) -> int:
         return run_nvpa_prefill(args, step, dev, lib, world, rank)
     work = decode_step_bytes(step)
     t = decode_to_device(step, dev)
+    if step.num_tokens > step.batch:
+        # a padded token list (slot -1 entries beyond the batch): the decode step takes one
+        # new row per sequence, the rows of the real tokens in sequence order
+        real = torch.as_tensor(np.nonzero(step.slot_mapping >= 0)[0][:step.batch], device=dev)
+        for k in ("k_new", "v_new", "slot_mapping"):
+            t[k] = t[k][real].contiguous()
     stream = torch.cuda.Stream(device=dev)
     shared = args.decode_api == "shared"
     if shared:
@@ -410,7 +415,10 @@ def run_nvpa(args) -> int:
     peaks = measured_peaks()
     value = work["step"] * world / (ms_step * 1e-3) / 1e9
     attn_gbs = work["step"] / (attn_ms * 1e-3) / 1e9
-    traffic = profile_traffic("decode_worker_b512", DECODE_SOURCES)
+    traffic = None
+    if args.workload == DEFAULT_WORKLOAD:
+        traffic = profile_traffic("decode_step_shared_prefix_b512" if shared else "decode_worker_b512",
+                                  DECODE_SOURCES)
     cs = clocks.summary()
     line = dict(
         metric=METRIC, value=value, unit="GB/s", n_gpus=world, steps=args.steps,
