@@ -238,7 +238,8 @@ size_t nvpa_decode_shared_prefix_workspace_size(int batch, int num_q_heads, int 
  *   workspace       at least nvpa_decode_shared_prefix_workspace_size(...) bytes,
  *                   256-byte aligned.  After the call its first 256 bytes hold int32
  *                   counters the plan wrote: [2] groups found, [3] sequences in them,
- *                   [4] prefix tile entries (diagnostics; read after the stream syncs).
+ *                   [4] prefix work units, each a pair of 128-row query tiles
+ *                   against one key partition (diagnostics; read after the stream syncs).
  *   other arguments as for nvpa_decode_step.
  * Errors: as nvpa_decode_step; a mix of NULL and non-NULL k_new/v_new/slot_mapping is
  * NVPA_ERR_INVALID_ARG.

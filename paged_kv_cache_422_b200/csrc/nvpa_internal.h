@@ -73,7 +73,7 @@ struct DecodePrefixArgs {
     int batch, hq, hkv, head_dim, num_blocks, block_size;
     float scale;
     int32_t* err_flag;
-    const int2* tiles;           // (group, query tile | partition << 16)
+    const int4* tiles;           // (group, query tile A, query tile B or -1, partition)
     const int32_t* ntiles;
     const int32_t* members;
     const int32_t* group_start;

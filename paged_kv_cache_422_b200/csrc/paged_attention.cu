@@ -68,7 +68,7 @@ struct AttnParams {
     int chunk, s_max;              // keys per partition, partitions of the longest context
     float scale_log2;
     // shared-prefix plan outputs (decode_plan_shared_kernel)
-    int2* ptiles;                  // (group, query tile | prefix partition << 16)
+    int4* ptiles;                  // (group, query tile A, query tile B or -1, prefix partition)
     int32_t* members;              // grouped member lists
     int32_t* group_start;          // [groups + 1]
     int32_t* group_len;            // [groups] prefix tokens
@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const AttnParams p) {
 //   private partitions npc .. npc+nsp-1 keys [prefix + s * chunk, ...), worker items;
 // and the combine merges all npc + nsp partials.  Sequences outside a group get the plain
 // decode plan's items.  Counters in the workspace: [0] next item, [1] items, [2] groups,
-// [3] members, [4] prefix tile entries.
+// [3] members, [4] prefix work units (pairs of query tiles of one group and partition).
 constexpr int kSharedTable = 2 * kSharedMaxBatch;   // a power of two above the batch
 
 __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& total) {
@@ -297,11 +297,15 @@ __global__ void __launch_bounds__(1024) decode_plan_shared_kernel(const AttnPara
         tlead[i] = 0;
         p.group_start[g] = m;
         p.group_len[g] = pre;
+        // query tiles of the group in pairs (the tensor-core kernel's work unit), for
+        // every prefix partition
         const int nq = (cnt + p.ptq - 1) / p.ptq;
+        const int npair = (nq + 1) / 2;
         const int nch = (pre + p.pchunk - 1) / p.pchunk;
-        const int off = atomicAdd(&s_ntiles, nq * nch);
+        const int off = atomicAdd(&s_ntiles, npair * nch);
         for (int c = 0; c < nch; ++c)
-            for (int qt = 0; qt < nq; ++qt) p.ptiles[off + c * nq + qt] = make_int2(g, qt | (c << 16));
+            for (int u = 0; u < npair; ++u)
+                p.ptiles[off + c * npair + u] = make_int4(g, 2 * u, 2 * u + 1 < nq ? 2 * u + 1 : -1, c);
         ++g;
         m += cnt;
     }
@@ -735,7 +739,7 @@ DecodeWorkspace decode_workspace_layout(int batch, int hq, int hkv, int head_dim
         w.members = off; off = align256(off + sizeof(int32_t) * (size_t)batch);
         w.group_start = off; off = align256(off + sizeof(int32_t) * ((size_t)batch + 1));
         w.group_len = off; off = align256(off + sizeof(int32_t) * (size_t)batch);
-        w.ptiles = off; off = align256(off + sizeof(int2) * (size_t)ptile_entries);
+        w.ptiles = off; off = align256(off + sizeof(int4) * (size_t)ptile_entries);
     }
     w.total = off;
     return w;
@@ -847,7 +851,7 @@ nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream) {
 
     cudaError_t e = cudaSuccess;
     if (shared) {
-        p.ptiles = reinterpret_cast<int2*>(ws + w.ptiles);
+        p.ptiles = reinterpret_cast<int4*>(ws + w.ptiles);
         p.members = reinterpret_cast<int32_t*>(ws + w.members);
         p.group_start = reinterpret_cast<int32_t*>(ws + w.group_start);
         p.group_len = reinterpret_cast<int32_t*>(ws + w.group_len);

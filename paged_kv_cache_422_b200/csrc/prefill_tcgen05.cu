@@ -1,40 +1,42 @@
-// Varlen causal prefill attention on the 5th-generation tensor cores (tcgen05 + TMEM).
+// Varlen causal prefill attention on the 5th-generation tensor cores (tcgen05 + TMEM),
+// and the same kernel in the shared-prefix mode of the decode step.
 //
 // ("Nano-vLLM inference engine architecture", section "Low-level performance details":
 // prefill runs a variable-length attention over cumulative sequence lengths; "Nano-vLLM
 // part 1" section 5.2 builds those lengths; section 4.2's prefix caching means the keys
 // of a sequence are its cached prefix followed by the suffix stored in this step.)
 //
-// Work unit: a tile of 128 query rows against one KV head.  The rows are 128/P tokens of
-// one sequence times the P query heads (P = query heads per KV head when that is a power
-// of two up to 8, else 1) that share the KV head, so each K/V tile fetched serves P
-// heads.  Keys come in tiles of 128 from the block-paged cache.  With a causal mask the
-// unit only visits key tiles up to its last token's position (bottom-right alignment:
-// suffix token r is at position Lk - Lq + r).
+// Query tile: 128 rows = 128/P tokens of one sequence times the P query heads (P = query
+// heads per KV head when that is a power of two up to 8, else 1) that share one KV head,
+// so each K/V tile fetched serves P heads.  Keys come in tiles of 128 from the
+// block-paged cache.  With a causal mask a query tile only visits key tiles up to its
+// last token's position (bottom-right alignment: suffix token r is at position
+// Lk - Lq + r).
 //
-// A one-CTA plan kernel lists the (sequence, query tile) pairs, longest first (by key
-// tiles visited).  The attention kernel is persistent with two CTAs per SM, so that one
-// CTA's softmax overlaps the other's MMAs; CTA c takes list entries c, c + gridDim.x, ...
-// for every KV head.  Inside a CTA the warps have roles:
-//   warp 0      TMA producer: the Q tile, then K_j and V_j tiles into a 2-stage ring
+// Work unit: a PAIR of query tiles of the same sequence and KV head (A = tile q, B = tile
+// q + 1, the one with more key tiles; B may be absent).  Both read the same K/V tiles, so
+// each tile is fetched once for 256 query rows, and the two tiles' MMAs and softmaxes
+// interleave: while one tile's softmax runs, the tensor core computes the other tile's
+// P V and its next S.  One CTA per SM (persistent; CTA c takes units c, c + grid, ...);
+// the plan kernel lists the pairs, heaviest sequences first.  Warp roles:
+//   warp 0      TMA producer: Q_A, Q_B, then K_j and V_j tiles into a 4-stage ring
 //               (one 3-D tensor-map box per cache block piece; a 128-key tile spans
 //               128 / block_size blocks when the block size is below 128);
-//   warp 1      allocates 256 TMEM columns; one lane issues the MMAs:
-//                 S_j = Q K_j^T   (SS: both operands in shared memory, K-major)
-//                 O  += P_j V_j   (TS: P from TMEM, V from shared memory, MN-major);
-//   warps 2..5  softmax, one thread per query row: read S_j from TMEM 32 columns at a
-//               time, mask, exponentiate against the current reference max, keep P_j
-//               packed in registers; only when some score exceeds the reference by more
-//               than 2^8 (always on the first tile) the reference moves, O is rescaled
-//               in TMEM and P_j is recomputed from S_j; then P_j is written as bf16 over
-//               S_j.  At the end O is divided by the row sum and stored with the lse.
-// TMEM columns: S/P [0, 128), O [128, 128 + D).  The MMAs of one thread execute in issue
-// order, so S_{j+1} (issued after O += P_j V_j) cannot overwrite P_j early.
+//   warp 1      allocates all 512 TMEM columns; one lane issues the MMAs in the order
+//                 S_A0 S_B0 | O_A += P_A0 V_0, S_A1, O_B += P_B0 V_0, S_B1 | ...
+//               where S = Q K_j^T is SS (both operands K-major in shared memory) and
+//               O += P V is TS (P from TMEM, V MN-major in shared memory);
+//   warps 2, 3  idle (they complete warpgroup 0, which gives registers to the softmax);
+//   warps 4..7  softmax of tile A, warps 8..11 softmax of tile B: one thread per query
+//               row (each warp on its own 32 TMEM lanes), see the pass comments below.
+// TMEM columns: tile A S/P [0, 128), O [128, 256); tile B S/P [256, 384), O [384, 512).
+// The MMAs of one thread execute in issue order, so S_{j+1} (issued after O += P_j V_j)
+// cannot overwrite P_j early.
 //
 // Stale rows (freed blocks are not cleared, part 1 section 4.3): K rows past the length
 // are masked in the softmax by select (never by arithmetic), and V rows past the length
-// in the last key tile are zeroed in shared memory before their MMA, so a 0 weight never
-// meets a NaN.
+// in the last key tile are zeroed in shared memory before their MMAs, so a 0 weight
+// never meets a NaN.
 #include <algorithm>
 #include <mutex>
 
@@ -50,10 +52,20 @@ namespace {
 
 constexpr int kQ = 128;          // query rows per tile (MMA M): tokens x packed heads
 constexpr int kKV = 128;         // keys per tile (MMA N of QK^T, K of PV)
-constexpr int kStages = 2;       // K/V ring stages, each one K or one V tile
-constexpr int kThreads = 192;    // 6 warps
-constexpr int kTmemCols = 256;   // S/P 128 + O up to 128
+constexpr int kStages = 4;       // K/V ring stages, each one K or one V tile
+constexpr int kWarps = 12;       // producer, MMA, 2 idle, 2 x 4 softmax
+constexpr int kThreads = kWarps * 32;
+// Register split (setmaxnreg acts on whole warpgroups): the launch gives every thread
+// kLaunchRegs; warpgroup 0 (producer, MMA, idle) gives registers back down to kSmallRegs
+// and the two softmax warpgroups take kSoftmaxRegs.  The shares add up to the launch's
+// total: 4 * kSmallRegs + 8 * kSoftmaxRegs == 12 * kLaunchRegs (per 32 lanes), and no
+// SM sub-partition (warps w, w+4, w+8) exceeds its 16384 registers.
+constexpr int kLaunchRegs = 168, kSmallRegs = 104, kSoftmaxRegs = 200;
+static_assert(4 * kSmallRegs + 8 * kSoftmaxRegs == 12 * kLaunchRegs, "register split");
+static_assert((kSmallRegs + 2 * kSoftmaxRegs) * 32 <= 16384, "sub-partition registers");
+constexpr int kTmemCols = 512;   // 2 tiles x (S/P 128 + O up to 128)
 constexpr int kMinTokensPerTile = 16;   // 128 rows / at most 8 packed heads
+
 // Bit k set for the first n of 32 columns (n clamped to [0, 32]).
 __device__ __forceinline__ uint32_t visible_mask(int n) {
     return n >= 32 ? 0xffffffffu : n <= 0 ? 0u : ((1u << n) - 1u);
@@ -147,7 +159,7 @@ struct PrefillParams {
     uint16_t* out;
     float* lse_out;
     int32_t* err;
-    const int2* tiles;           // plan: (sequence, query tile), longest first
+    const int4* tiles;           // plan: (sequence, query tile A, query tile B or -1, key partition)
     const int32_t* ntiles;       // plan: number of entries
     // shared-prefix decode mode: "sequences" are prefix groups whose "queries" are the
     // members' decode query rows; results go to each member's prefix partition slot
@@ -173,20 +185,21 @@ struct Layout {
     static constexpr int REGIONS = D / 64;                  // 64 bf16 = one 128-byte swizzle row
     static constexpr int REGION_BYTES = 128 * 128;          // 128 rows x 128 bytes
     static constexpr int TILE_BYTES = REGIONS * REGION_BYTES;
-    static constexpr int Q_OFF = 0;
-    static constexpr int STAGE_OFF = TILE_BYTES;
+    static constexpr int Q_OFF = 0;                         // Q_A, Q_B
+    static constexpr int STAGE_OFF = 2 * TILE_BYTES;
     static constexpr int BAR_OFF = STAGE_OFF + kStages * TILE_BYTES;
-    // barriers
-    static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_KVFULL = 2, B_KVEMPTY = B_KVFULL + kStages;
-    static constexpr int B_SFULL = B_KVEMPTY + kStages, B_PFULL = B_SFULL + 1;
-    static constexpr int B_ODONE = B_PFULL + 1, B_OFINAL = B_ODONE + 1, B_OFREE = B_OFINAL + 1;
-    static constexpr int B_DRAIN = B_OFREE + 1, NBARS = B_DRAIN + 1;
+    // barriers (the per-tile ones come in pairs: + 0 for tile A, + 1 for tile B)
+    static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KVFULL = 4, B_KVEMPTY = B_KVFULL + kStages;
+    static constexpr int B_SFULL = B_KVEMPTY + kStages, B_PFULL = B_SFULL + 2, B_ODONE = B_PFULL + 2;
+    static constexpr int B_OFINAL = B_ODONE + 2, B_OFREE = B_OFINAL + 2, B_DRAIN = B_OFREE + 2;
+    static constexpr int NBARS = B_DRAIN + 1;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;     // tmem base, abort flag
     static constexpr int BYTES = MISC_OFF + 16;
     static constexpr int ALLOC = BYTES + 1024;               // room to align the base to 1024
 };
 
 struct TileInfo {
+    bool valid;          // false: the pair's B slot is empty
     int seq, qt, head0, hk;
     int q0, lq, lk;      // first query row (global), query rows, keys of the sequence
     int kbeg, chunk;     // shared-prefix mode: first key and index of the key partition
@@ -199,18 +212,20 @@ __device__ __forceinline__ int tile_nkv(int causal, int lq, int lk, int tok0, in
     return causal ? min(ktiles, (lk - lq + tok0 + ntok - 1) / kKV + 1) : ktiles;
 }
 
+// Tile A (second = false) or B of plan entry e for head group hg.
 template <bool PREFIX>
-__device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, int idx) {
+__device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, int4 e, int hg, bool second) {
     TileInfo t;
-    const int2 e = __ldg(p.tiles + idx / p.hgroups);
+    const int qt = second ? e.z : e.y;
+    t.valid = qt >= 0;
     t.seq = e.x;
-    t.qt = e.y & 0xffff;
-    t.head0 = (idx % p.hgroups) * p.pack;
+    t.qt = max(qt, 0);
+    t.head0 = hg * p.pack;
     t.hk = t.head0 / p.group;
     if constexpr (PREFIX) {
         // group e.x: its members are the queries, keys [kbeg, kbeg + lk) of its shared
         // prefix the keys (no mask)
-        t.chunk = e.y >> 16;
+        t.chunk = e.w;
         t.kbeg = t.chunk * p.pchunk;
         t.q0 = __ldg(p.group_start + t.seq);
         t.lq = __ldg(p.group_start + t.seq + 1) - t.q0;
@@ -224,20 +239,29 @@ __device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, int idx) {
     }
     t.tok0 = t.qt * p.tq;
     t.ntok = min(p.tq, t.lq - t.tok0);
-    t.nkv = tile_nkv(PREFIX ? 0 : p.causal, t.lq, t.lk, t.tok0, t.ntok);
+    t.nkv = t.valid ? tile_nkv(PREFIX ? 0 : p.causal, t.lq, t.lk, t.tok0, t.ntok) : 0;
     return t;
 }
 
 // ------------------------------------------------------------------------------------
-// plan: list (sequence, query tile) pairs, most key tiles first
+// plan: list the query-tile pairs, the sequences with the most key tiles first
 // ------------------------------------------------------------------------------------
 constexpr int kPlanMaxRanked = 2048;   // batches up to this size are ordered by sequence
 
 // Entries are grouped by sequence, sequences with the most work (key tiles visited over
-// all their query tiles) first and, inside a sequence, query tiles with the most key
-// tiles first.  CTAs that run at the same time then mostly read the same sequences' keys
-// and values, which L2 serves after the first fetch, and the longest work starts first.
-__global__ void __launch_bounds__(1024) prefill_plan_kernel(const PrefillParams p, int2* tiles,
+// all their query tiles) first and, inside a sequence, the pairs with the most key tiles
+// first.  CTAs that run at the same time then mostly read the same sequences' keys and
+// values, which L2 serves after the first fetch, and the longest work starts first.  A
+// sequence with cnt query tiles gives the pairs (cnt-2, cnt-1), (cnt-4, cnt-3), ... and,
+// for odd cnt, the single tile 0.
+__device__ __forceinline__ void write_pairs(int4* tiles, int off, int seq, int cnt) {
+    for (int u = 0; 2 * u < cnt; ++u) {
+        const int b = cnt - 1 - 2 * u;
+        tiles[off + u] = b >= 1 ? make_int4(seq, b - 1, b, 0) : make_int4(seq, 0, -1, 0);
+    }
+}
+
+__global__ void __launch_bounds__(1024) prefill_plan_kernel(const PrefillParams p, int4* tiles,
                                                             int32_t* ntiles) {
     __shared__ int s_work[kPlanMaxRanked];
     __shared__ int s_count[kPlanMaxRanked];
@@ -253,7 +277,7 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const PrefillParams 
                q1 <= p.total_q;
     };
     const int nb = min(p.batch, kPlanMaxRanked);
-    // per sequence: tiles and work (0 tiles for a malformed sequence, which is flagged)
+    // per sequence: pairs and work (nothing for a malformed sequence, which is flagged)
     for (int i = tid; i < kPlanMaxRanked; i += blockDim.x) {
         int lq = 0, lk = 0, cnt = 0, work = 0;
         if (i < p.batch) {
@@ -267,7 +291,7 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const PrefillParams 
         }
         if (i < nb) {
             s_work[i] = work;
-            s_count[i] = cnt;
+            s_count[i] = (cnt + 1) / 2;
         }
     }
     __syncthreads();
@@ -286,7 +310,7 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const PrefillParams 
         rank_of[k] = rnk;
     }
     __syncthreads();
-    // reorder the tile counts by rank (reuse s_work as counts-in-rank-order)
+    // reorder the pair counts by rank (reuse s_work as counts-in-rank-order)
     for (int k = 0; k < kPlanMaxRanked / 1024; ++k) {
         const int i = tid + k * 1024;
         if (i < nb) s_work[rank_of[k]] = s_count[i];
@@ -323,15 +347,12 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const PrefillParams 
     }
     __syncthreads();
     int written = carry;
-    // write each ranked sequence's tiles, most key tiles (last query tile) first
     for (int k = 0; k < kPlanMaxRanked / 1024; ++k) {
         const int i = tid + k * 1024;
         if (i >= nb) continue;
         int lq, lk;
         if (!seq_ok(i, lq, lk)) continue;
-        const int cnt = (lq + p.tq - 1) / p.tq;
-        const int off = s_count[rank_of[k]];
-        for (int u = 0; u < cnt; ++u) tiles[off + u] = make_int2(i, cnt - 1 - u);
+        write_pairs(tiles, s_count[rank_of[k]], i, (lq + p.tq - 1) / p.tq);
     }
     // sequences beyond the ranked ones (very large batches) follow in index order
     if (p.batch > nb) {
@@ -342,8 +363,7 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const PrefillParams 
             int lq, lk;
             if (!seq_ok(i, lq, lk)) continue;
             const int cnt = (lq + p.tq - 1) / p.tq;
-            const int off = atomicAdd(&extra_base, cnt);
-            for (int u = 0; u < cnt; ++u) tiles[off + u] = make_int2(i, cnt - 1 - u);
+            write_pairs(tiles, atomicAdd(&extra_base, (cnt + 1) / 2), i, cnt);
         }
         __syncthreads();
         if (tid == 0) written = extra_base;
@@ -355,7 +375,7 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const PrefillParams 
 // the attention kernel
 // ------------------------------------------------------------------------------------
 template <int D, bool PREFIX>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
 prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap k_map,
                        const __grid_constant__ CUtensorMap v_map, const PrefillParams p) {
     using L = Layout<D>;
@@ -377,17 +397,19 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
     }
 
     if (threadIdx.x == 0) {
-        mbar_init(bars + L::B_QFULL, 1);
-        mbar_init(bars + L::B_QEMPTY, 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(bars + L::B_QFULL + x, 1);
+            mbar_init(bars + L::B_QEMPTY + x, 1);
+            mbar_init(bars + L::B_SFULL + x, 1);
+            mbar_init(bars + L::B_PFULL + x, 4);
+            mbar_init(bars + L::B_ODONE + x, 1);
+            mbar_init(bars + L::B_OFINAL + x, 1);
+            mbar_init(bars + L::B_OFREE + x, 4);
+        }
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bars + L::B_KVFULL + s, 1);
             mbar_init(bars + L::B_KVEMPTY + s, 1);
         }
-        mbar_init(bars + L::B_SFULL, 1);
-        mbar_init(bars + L::B_PFULL, 4);
-        mbar_init(bars + L::B_ODONE, 1);
-        mbar_init(bars + L::B_OFINAL, 1);
-        mbar_init(bars + L::B_OFREE, 4);
         mbar_init(bars + L::B_DRAIN, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -403,17 +425,19 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t TM_S = 0, TM_O = kKV;   // column offsets
 
     const int total = __ldcg(p.ntiles) * p.hgroups;
 
-    if (warp == 0) {
+    if (warp < 4) {
+      // warpgroup 0: producer, MMA issuer and two idle warps, with few registers
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kSmallRegs));
+      if (warp == 0) {
         // ============================ TMA producer ============================
-        // The whole warp walks the tiles; lane 0 issues the copies and barrier operations,
+        // The whole warp walks the units; lane 0 issues the copies and barrier operations,
         // lane c < 8 holds the physical block of piece c of the next key tile, loaded one
         // key tile ahead so that no copy waits on a block-table lookup.
         uint32_t fill = 0;
-        int tcount = 0;
+        int qloads[2] = {0, 0};
         int last_fill[kStages];
         for (int s = 0; s < kStages; ++s) last_fill[s] = -1;
         const int piece = min(p.block_size, kKV);
@@ -430,53 +454,66 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             }
             return blk;
         };
-        for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
-            const TileInfo t = tile_info<PREFIX>(p, idx);
-            const int bt_seq = PREFIX ? __ldg(p.members + t.q0) : t.seq;   // a member's table
+        bool ok = true;
+        for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
+            const int4 e = __ldg(p.tiles + idx / p.hgroups);
+            const int hg = idx % p.hgroups;
+            const TileInfo ta = tile_info<PREFIX>(p, e, hg, false);
+            const TileInfo tb = tile_info<PREFIX>(p, e, hg, true);
+            const int nkv = max(ta.nkv, tb.nkv);
+            const int bt_seq = PREFIX ? __ldg(p.members + ta.q0) : ta.seq;   // a member's table
             const int32_t* bt = p.block_tables + (size_t)bt_seq * p.max_blocks;
-            int cur_blk = load_pieces(bt, t.kbeg, t.lk, 0);
-            if (!mbar_wait(bars + L::B_QEMPTY, (tcount & 1) ^ 1, abort_flag, p.err)) break;
-            if constexpr (PREFIX) {
-                // gather the members' query rows into the swizzled Q tile with 16-byte
-                // cp.async copies, all in flight at once: lane l fills rows l, l+32, l+64,
-                // l+96; row r is member tok0 + r / P, head head0 + r % P, and 16-byte chunk c
-                // of its 128-byte half goes to chunk c ^ (r % 8) (the 128-byte swizzle the
-                // MMA descriptors expect).  Rows past the group are zero-filled.
-                const uint16_t* src[kQ / 32];
-#pragma unroll
-                for (int i = 0; i < kQ / 32; ++i) {
-                    const int r = lane + 32 * i;
-                    const int mi = t.tok0 + (r >> p.pack_shift);
-                    const int b = mi < t.lq ? __ldg(p.members + t.q0 + mi) : -1;
-                    src[i] = b < 0 ? nullptr
-                                   : p.q_rows + ((size_t)b * p.hq + t.head0 + (r & (p.pack - 1))) * D;
+            int cur_blk = load_pieces(bt, ta.kbeg, ta.lk, 0);
+            for (int x = 0; x < 2 && ok; ++x) {
+                const TileInfo& t = x ? tb : ta;
+                if (!t.valid) continue;
+                if (!mbar_wait(bars + L::B_QEMPTY + x, (qloads[x] & 1) ^ 1, abort_flag, p.err)) {
+                    ok = false;
+                    break;
                 }
+                uint8_t* qdst = smem + L::Q_OFF + x * L::TILE_BYTES;
+                if constexpr (PREFIX) {
+                    // gather the members' query rows into the swizzled Q tile with 16-byte
+                    // cp.async copies, all in flight at once: lane l fills rows l, l+32,
+                    // l+64, l+96; row r is member tok0 + r / P, head head0 + r % P, and
+                    // 16-byte chunk c of its 128-byte half goes to chunk c ^ (r % 8) (the
+                    // 128-byte swizzle the MMA descriptors expect).  Rows past the group
+                    // are zero-filled.
+                    const uint16_t* src[kQ / 32];
 #pragma unroll
-                for (int i = 0; i < kQ / 32; ++i) {
-                    const int r = lane + 32 * i;
+                    for (int i = 0; i < kQ / 32; ++i) {
+                        const int r = lane + 32 * i;
+                        const int mi = t.tok0 + (r >> p.pack_shift);
+                        const int b = mi < t.lq ? __ldg(p.members + t.q0 + mi) : -1;
+                        src[i] = b < 0 ? nullptr
+                                       : p.q_rows + ((size_t)b * p.hq + t.head0 + (r & (p.pack - 1))) * D;
+                    }
 #pragma unroll
-                    for (int c = 0; c < D / 8; ++c) {
-                        uint8_t* dst = smem + L::Q_OFF + (c / 8) * L::REGION_BYTES + r * 128 +
-                                       (((c % 8) ^ (r & 7)) * 16);
-                        cp_async16(dst, src[i] != nullptr ? src[i] + c * 8 : p.q_rows, src[i] != nullptr ? 16 : 0);
+                    for (int i = 0; i < kQ / 32; ++i) {
+                        const int r = lane + 32 * i;
+#pragma unroll
+                        for (int c = 0; c < D / 8; ++c) {
+                            uint8_t* dst = qdst + (c / 8) * L::REGION_BYTES + r * 128 + (((c % 8) ^ (r & 7)) * 16);
+                            cp_async16(dst, src[i] != nullptr ? src[i] + c * 8 : p.q_rows, src[i] != nullptr ? 16 : 0);
+                        }
+                    }
+                    cp_async_commit();
+                    cp_async_wait<0>();
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bars + L::B_QFULL + x);
+                } else {
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(bars + L::B_QFULL + x, L::TILE_BYTES);
+                        for (int r = 0; r < L::REGIONS; ++r)
+                            tma_load_3d(qdst + r * L::REGION_BYTES, &q_map, bars + L::B_QFULL + x, r * 64,
+                                        t.head0, t.q0 + t.tok0);
                     }
                 }
-                cp_async_commit();
-                cp_async_wait<0>();
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bars + L::B_QFULL);
-            } else {
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(bars + L::B_QFULL, L::TILE_BYTES);
-                    for (int r = 0; r < L::REGIONS; ++r)
-                        tma_load_3d(smem + L::Q_OFF + r * L::REGION_BYTES, &q_map, bars + L::B_QFULL, r * 64,
-                                    t.head0, t.q0 + t.tok0);
-                }
+                ++qloads[x];
             }
-            bool ok = true;
-            for (int j = 0; j < t.nkv && ok; ++j) {
-                const int nxt_blk = j + 1 < t.nkv ? load_pieces(bt, t.kbeg, t.lk, j + 1) : -1;
+            for (int j = 0; j < nkv && ok; ++j) {
+                const int nxt_blk = j + 1 < nkv ? load_pieces(bt, ta.kbeg, ta.lk, j + 1) : -1;
                 const int key0 = j * kKV;
                 const uint32_t valid_mask = __ballot_sync(0xffffffffu, cur_blk >= 0);
                 const uint32_t bytes = (uint32_t)__popc(valid_mask) * (uint32_t)(piece * 128 * L::REGIONS);
@@ -493,11 +530,11 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                         const int c = __ffs(m) - 1;
                         const int blk = __shfl_sync(0xffffffffu, cur_blk, c);
                         if (lane == 0) {
-                            const int kc = t.kbeg + key0 + c * piece;
+                            const int kc = ta.kbeg + key0 + c * piece;
                             const int z = blk * p.block_size + (kc & (p.block_size - 1));
                             for (int r = 0; r < L::REGIONS; ++r)
                                 tma_load_3d(dst + r * L::REGION_BYTES + c * piece * 128, map,
-                                            bars + L::B_KVFULL + slot, r * 64, t.hk, z);
+                                            bars + L::B_KVFULL + slot, r * 64, ta.hk, z);
                         }
                     }
                     last_fill[slot] = (int)fill;
@@ -505,8 +542,6 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                 }
                 cur_blk = nxt_blk;
             }
-            ++tcount;
-            if (!ok) break;
         }
         // let every copy this warp started land before the CTA can exit
         if (lane == 0) {
@@ -517,60 +552,80 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                        global_ns() - t0 < 100000000ull) {
                 }
             }
-            if (tcount > 0) {
+            for (int x = 0; x < 2; ++x) {
+                if (qloads[x] == 0) continue;
                 const uint64_t t0 = global_ns();
-                while (!mbar_try_wait(bars + L::B_QFULL, (tcount - 1) & 1) && global_ns() - t0 < 100000000ull) {
+                while (!mbar_try_wait(bars + L::B_QFULL + x, (qloads[x] - 1) & 1) && global_ns() - t0 < 100000000ull) {
                 }
             }
         }
-    } else if (warp == 1) {
+      } else if (warp == 1) {
         // ============================ MMA issuer ============================
+        // Per unit: S_A0, S_B0, then for each key tile j: O_A += P_Aj V_j, S_A(j+1),
+        // O_B += P_Bj V_j, S_B(j+1).  Tile A's softmax of key tile j+1 thus overlaps tile
+        // B's P V and S MMAs, and the other way round.  K_j's ring slot is released after
+        // the last S that reads it, V_j's after the last P V.
         constexpr uint32_t IDESC_QK = idesc_bf16_f32(kQ, kKV, false);
         constexpr uint32_t IDESC_PV = idesc_bf16_f32(kQ, D, true);
-        const uint32_t q_addr = sbase + L::Q_OFF;
-        uint32_t fbase = 0;   // ring fill index of this tile's K_0 (K_j = fbase + 2j, V_j = +1)
-        int tcount = 0;
-        uint32_t p_use = 0;
+        uint32_t fbase = 0;                    // ring fill index of this unit's K_0
+        int quse[2] = {0, 0};                  // Q tiles consumed per slot
+        uint32_t puse[2] = {0, 0};             // P_j waits per tile
+        int units[2] = {0, 0};                 // units in which the tile had work
         bool ok = true;
-        for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
-            const TileInfo t = tile_info<PREFIX>(p, idx);
-            if (!mbar_wait(bars + L::B_QFULL, tcount & 1, abort_flag, p.err)) break;
-            for (int j = 0; j < t.nkv && ok; ++j) {
-                // S_j = Q K_j^T
-                const uint32_t fk = fbase + 2 * (uint32_t)j;
-                const int kslot = fk % kStages;
-                if (!mbar_wait(bars + L::B_KVFULL + kslot, (fk / kStages) & 1, abort_flag, p.err)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t k_addr = sbase + L::STAGE_OFF + kslot * L::TILE_BYTES;
+        auto issue_qk = [&](int x, int kslot) {
+            const uint32_t q_addr = sbase + L::Q_OFF + x * L::TILE_BYTES;
+            const uint32_t k_addr = sbase + L::STAGE_OFF + kslot * L::TILE_BYTES;
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const int r = kk / 4, off = (kk % 4) * 32;
-                        const uint64_t adesc = sdesc_sw128(q_addr + r * L::REGION_BYTES + off, 16, 1024);
-                        const uint64_t bdesc = sdesc_sw128(k_addr + r * L::REGION_BYTES + off, 16, 1024);
-                        umma_ss(tmem + TM_S, adesc, bdesc, IDESC_QK, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(bars + L::B_KVEMPTY + kslot);
-                    umma_commit(bars + L::B_SFULL);
-                    if (j == t.nkv - 1) umma_commit(bars + L::B_QEMPTY);
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const int r = kk / 4, off = (kk % 4) * 32;
+                const uint64_t adesc = sdesc_sw128(q_addr + r * L::REGION_BYTES + off, 16, 1024);
+                const uint64_t bdesc = sdesc_sw128(k_addr + r * L::REGION_BYTES + off, 16, 1024);
+                umma_ss(tmem + x * 256, adesc, bdesc, IDESC_QK, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(bars + L::B_SFULL + x);
+        };
+        auto issue_pv = [&](int x, int vslot, bool accumulate) {
+            const uint32_t v_addr = sbase + L::STAGE_OFF + vslot * L::TILE_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < kKV / 16; ++kk) {
+                const uint64_t bdesc = sdesc_sw128(v_addr + kk * 16 * 128, L::REGION_BYTES, 1024);
+                umma_ts(tmem + x * 256 + kKV, tmem + x * 256 + kk * 8, bdesc, IDESC_PV,
+                        (accumulate || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(bars + L::B_ODONE + x);
+        };
+        for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
+            const int4 e = __ldg(p.tiles + idx / p.hgroups);
+            const int hg = idx % p.hgroups;
+            const TileInfo ta = tile_info<PREFIX>(p, e, hg, false);
+            const TileInfo tb = tile_info<PREFIX>(p, e, hg, true);
+            const int nk[2] = {ta.nkv, tb.nkv};
+            const bool val[2] = {ta.valid, tb.valid};
+            const int nkv = max(nk[0], nk[1]);
+            for (int x = 0; x < 2 && ok; ++x)
+                if (val[x] && !mbar_wait(bars + L::B_QFULL + x, quse[x] & 1, abort_flag, p.err)) ok = false;
+            if (!ok) break;
+            if (nkv > 0) {
+                const int kslot = fbase % kStages;
+                if (!mbar_wait(bars + L::B_KVFULL + kslot, (fbase / kStages) & 1, abort_flag, p.err)) break;
+            }
+            tc_fence_after();
+            if (lane == 0) {
+                for (int x = 0; x < 2; ++x) {
+                    if (nk[x] > 0) issue_qk(x, fbase % kStages);
+                    if (val[x] && nk[x] <= 1) umma_commit(bars + L::B_QEMPTY + x);
                 }
-                __syncwarp();
-                // O += P_j V_j
-                if (!mbar_wait(bars + L::B_PFULL, p_use & 1, abort_flag, p.err)) {
-                    ok = false;
-                    break;
-                }
-                ++p_use;
-                const uint32_t fv = fk + 1;
-                const int vslot = fv % kStages;
+                if (nkv > 0) umma_commit(bars + L::B_KVEMPTY + fbase % kStages);
+            }
+            __syncwarp();
+            for (int j = 0; j < nkv && ok; ++j) {
+                const uint32_t fv = fbase + 2 * (uint32_t)j + 1, fk = fv + 1;
+                const int vslot = fv % kStages, kslot = fk % kStages;
                 if (!mbar_wait(bars + L::B_KVFULL + vslot, (fv / kStages) & 1, abort_flag, p.err)) {
                     ok = false;
                     break;
                 }
-                const int valid = min(kKV, t.lk - j * kKV);
+                const int valid = min(kKV, ta.lk - j * kKV);
                 if (valid < kKV) {
                     // zero the V rows past the sequence (stale cache rows, or never loaded)
                     uint8_t* vt = smem + L::STAGE_OFF + vslot * L::TILE_BYTES;
@@ -582,28 +637,49 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                     fence_proxy_async_smem();
                     __syncwarp();
                 }
-                if (j == 0 && tcount > 0) {
-                    if (!mbar_wait(bars + L::B_OFREE, (tcount - 1) & 1, abort_flag, p.err)) {
+                bool k_next = false;
+                for (int x = 0; x < 2; ++x) {
+                    if (j >= nk[x]) continue;
+                    if (!mbar_wait(bars + L::B_PFULL + x, puse[x] & 1, abort_flag, p.err)) {
                         ok = false;
                         break;
                     }
-                }
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t v_addr = sbase + L::STAGE_OFF + vslot * L::TILE_BYTES;
-#pragma unroll
-                    for (int kk = 0; kk < kKV / 16; ++kk) {
-                        const uint64_t bdesc = sdesc_sw128(v_addr + kk * 16 * 128, L::REGION_BYTES, 1024);
-                        umma_ts(tmem + TM_O, tmem + TM_S + kk * 8, bdesc, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+                    ++puse[x];
+                    if (j == 0 && units[x] > 0 &&
+                        !mbar_wait(bars + L::B_OFREE + x, (units[x] - 1) & 1, abort_flag, p.err)) {
+                        ok = false;
+                        break;
                     }
+                    if (j + 1 < nk[x] && !k_next) {
+                        if (!mbar_wait(bars + L::B_KVFULL + kslot, (fk / kStages) & 1, abort_flag, p.err)) {
+                            ok = false;
+                            break;
+                        }
+                        k_next = true;
+                    }
+                    tc_fence_after();
+                    if (lane == 0) {
+                        issue_pv(x, vslot, j > 0);
+                        if (j == nk[x] - 1) umma_commit(bars + L::B_OFINAL + x);
+                        if (j + 1 < nk[x]) {
+                            issue_qk(x, kslot);
+                            if (j + 2 == nk[x]) umma_commit(bars + L::B_QEMPTY + x);
+                        }
+                    }
+                    __syncwarp();
+                }
+                if (!ok) break;
+                if (lane == 0) {
                     umma_commit(bars + L::B_KVEMPTY + vslot);
-                    umma_commit(bars + L::B_ODONE);
-                    if (j == t.nkv - 1) umma_commit(bars + L::B_OFINAL);
+                    if (k_next) umma_commit(bars + L::B_KVEMPTY + kslot);
                 }
                 __syncwarp();
             }
-            fbase += 2 * (uint32_t)t.nkv;
-            ++tcount;
+            fbase += 2 * (uint32_t)nkv;
+            for (int x = 0; x < 2; ++x) {
+                if (val[x]) ++quse[x];
+                if (nk[x] > 0) ++units[x];
+            }
         }
         // every MMA this thread issued completes before TMEM is released
         if (lane == 0) umma_commit(bars + L::B_DRAIN);
@@ -611,27 +687,37 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
         const uint64_t t0 = global_ns();
         while (!mbar_try_wait(bars + L::B_DRAIN, 0) && global_ns() - t0 < 100000000ull) {
         }
+      }
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
         // ============================ softmax warps ============================
+        // warps 4..7: tile A, warps 8..11: tile B
+        const int x = (warp - 4) >> 2;
         const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
         const int r = quarter * 32 + lane;            // row of the tile: token r / P, head r % P
         const int rtok = r >> p.pack_shift;
         const int rhead = r & (p.pack - 1);
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-        const uint32_t s_col = tmem + lane_base + TM_S;
-        const uint32_t o_col = tmem + lane_base + TM_O;
+        const uint32_t s_col = tmem + lane_base + x * 256;
+        const uint32_t o_col = s_col + kKV;
+        uint64_t* b_sfull = bars + L::B_SFULL + x;
+        uint64_t* b_pfull = bars + L::B_PFULL + x;
+        uint64_t* b_odone = bars + L::B_ODONE + x;
+        uint64_t* b_ofinal = bars + L::B_OFINAL + x;
+        uint64_t* b_ofree = bars + L::B_OFREE + x;
         uint32_t s_use = 0;
         int tcount = 0;
-        uint32_t pv_before = 0;                       // PVs issued for earlier tiles
+        uint32_t pv_before = 0;                       // PVs issued for this tile slot before
         for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
-            const TileInfo t = tile_info<PREFIX>(p, idx);
+            const TileInfo t = tile_info<PREFIX>(p, __ldg(p.tiles + idx / p.hgroups), idx % p.hgroups, x == 1);
+            if (t.nkv == 0) continue;
             const int pos = t.lk - t.lq + t.tok0 + rtok;           // absolute position of this row
             const int lim = (!PREFIX && p.causal) ? min(t.lk, pos + 1) : t.lk;  // keys 0 .. lim-1 visible
             const int lim_min = __reduce_min_sync(0xffffffffu, lim);
             float m = -INFINITY, l = 0.f;
             bool ok = true;
             for (int j = 0; j < t.nkv; ++j) {
-                if (!mbar_wait(bars + L::B_SFULL, s_use & 1, abort_flag, p.err)) {
+                if (!mbar_wait(b_sfull, s_use & 1, abort_flag, p.err)) {
                     ok = false;
                     break;
                 }
@@ -675,7 +761,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                 if (rescale && j > 0) {
                     // O holds P_0..P_{j-1} V (all complete once S_j is): rescale it before
                     // P_j is released to the MMA
-                    if (!mbar_wait(bars + L::B_ODONE, (pv_before + j - 1) & 1, abort_flag, p.err)) {
+                    if (!mbar_wait(b_odone, (pv_before + j - 1) & 1, abort_flag, p.err)) {
                         ok = false;
                         break;
                     }
@@ -693,10 +779,10 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bars + L::B_PFULL);
+                if (lane == 0) mbar_arrive(b_pfull);
             }
             if (!ok) break;
-            if (!mbar_wait(bars + L::B_OFINAL, tcount & 1, abort_flag, p.err)) break;
+            if (!mbar_wait(b_ofinal, tcount & 1, abort_flag, p.err)) break;
             tc_fence_after();
             const bool row_ok = rtok < t.ntok;
             const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -718,7 +804,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                 if (c == D / 32 - 1) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(bars + L::B_OFREE);
+                    if (lane == 0) mbar_arrive(b_ofree);
                 }
                 if (PREFIX && row_ok) {
 #pragma unroll
@@ -862,7 +948,7 @@ cudaError_t launch_decode_prefix_tcgen05(const DecodePrefixArgs& a, cudaStream_t
     p.block_shift = __builtin_ctz((unsigned)a.block_size);
     p.scale_log2 = a.scale * kLog2e;
     const long long units = std::max(1LL, a.max_entries) * p.hgroups;
-    const long long cap = a.max_ctas > 0 ? a.max_ctas : 2LL * device_sm_count();
+    const long long cap = a.max_ctas > 0 ? a.max_ctas : (long long)device_sm_count();
     const int grid = (int)std::max(1LL, std::min<long long>(cap, units));
     // the query map is not read in this mode (rows are gathered); any valid map will do
     return a.head_dim == 128 ? launch_prefill<128, true>(km, km, vm, p, grid, stream, a.pdl)
@@ -872,7 +958,7 @@ cudaError_t launch_decode_prefix_tcgen05(const DecodePrefixArgs& a, cudaStream_t
 size_t prefill_workspace_bytes(int batch, int total_q) {
     const size_t entries = (size_t)std::max(0, batch) +
                            ((size_t)std::max(0, total_q) + kMinTokensPerTile - 1) / kMinTokensPerTile;
-    return 256 + ((entries * sizeof(int2) + 255) & ~size_t(255));
+    return 256 + ((entries * sizeof(int4) + 255) & ~size_t(255));
 }
 
 nvpa_status_t run_varlen_prefill_tcgen05(const PrefillCall& c, void* workspace, size_t workspace_bytes,
@@ -902,7 +988,7 @@ nvpa_status_t run_varlen_prefill_tcgen05(const PrefillCall& c, void* workspace, 
     p.lse_out = c.lse_out;
     p.err = c.err_flag;
     p.ntiles = reinterpret_cast<int32_t*>(ws);
-    p.tiles = reinterpret_cast<int2*>(ws + 256);
+    p.tiles = reinterpret_cast<const int4*>(ws + 256);
     p.batch = c.batch;
     p.total_q = c.total_q;
     p.hq = c.hq;
@@ -921,12 +1007,13 @@ nvpa_status_t run_varlen_prefill_tcgen05(const PrefillCall& c, void* workspace, 
     p.causal = c.causal;
     p.scale_log2 = c.scale * kLog2e;
 
-    prefill_plan_kernel<<<1, 1024, 0, stream>>>(p, reinterpret_cast<int2*>(ws + 256), reinterpret_cast<int32_t*>(ws));
+    prefill_plan_kernel<<<1, 1024, 0, stream>>>(p, reinterpret_cast<int4*>(ws + 256), reinterpret_cast<int32_t*>(ws));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_failure(e, "prefill plan launch");
     count_launches(1);
-    const long long max_tiles = ((long long)c.batch + (c.total_q + p.tq - 1) / p.tq) * p.hgroups;
-    const int grid = (int)std::max(1LL, std::min<long long>(2LL * device_sm_count(), max_tiles));
+    // one pair per query tile at most, plus one per sequence for a ragged last tile
+    const long long max_units = ((long long)c.batch + (c.total_q + p.tq - 1) / p.tq) * p.hgroups;
+    const int grid = (int)std::max(1LL, std::min<long long>((long long)device_sm_count(), max_units));
     e = c.head_dim == 128 ? launch_prefill<128, false>(qm, km, vm, p, grid, stream)
                           : launch_prefill<64, false>(qm, km, vm, p, grid, stream);
     if (e != cudaSuccess) return cuda_failure(e, "prefill tcgen05 launch");

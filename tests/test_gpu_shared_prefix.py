@@ -85,8 +85,9 @@ def test_batch512_shared_prefix_workload(cuda_device):
     (groups, members, tiles), _, _ = _run(step, cuda_device, seqs=seqs)
     assert groups == 1
     assert members == int(shared.sum())
-    # 1024 prefix keys in 4 partitions of 256; 64 members per tile (2 query heads a row pair)
-    assert tiles == 4 * ((members + 63) // 64)
+    # 1024 prefix keys in 4 partitions of 256; 64 members per query tile (2 query heads
+    # each), query tiles in pairs
+    assert tiles == 4 * (((members + 63) // 64 + 1) // 2)
 
 
 @pytest.mark.parametrize("store", [True, False])
@@ -110,7 +111,7 @@ def test_shared_prefix_shapes(cuda_device, lens, hq, hkv, d, bs, nshared, nblk, 
     (groups, members, tiles), _, _ = _run(step, cuda_device, store=store, min_group=4)
     assert (groups, members) == (1, nshared)
     tq = 128 // (hq // hkv if (hq // hkv) & (hq // hkv - 1) == 0 else 1)
-    assert tiles == -(-nblk * bs // 256) * -(-nshared // tq)
+    assert tiles == -(-nblk * bs // 256) * ((-(-nshared // tq) + 1) // 2)   # query-tile pairs
 
 
 def test_two_groups_and_a_short_common_run(cuda_device):
@@ -124,7 +125,7 @@ def test_two_groups_and_a_short_common_run(cuda_device):
     step.block_tables[19, 2:4] = step.block_tables[20, 2:4]   # 19: common run of 2
     (groups, members, tiles), _, _ = _run(step, cuda_device, min_group=4)
     assert (groups, members) == (2, 20)
-    assert tiles == 1 + 1      # one query tile and one partition each (160 and 64 keys)
+    assert tiles == 1 + 1      # one query tile (pair) and one partition each (160 and 64 keys)
 
 
 def test_member_whose_private_part_is_its_new_token(cuda_device):
