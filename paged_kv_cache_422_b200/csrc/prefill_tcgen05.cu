@@ -19,9 +19,11 @@
 // interleave: while one tile's softmax runs, the tensor core computes the other tile's
 // P V and its next S.  One CTA per SM (persistent; CTA c takes units c, c + grid, ...);
 // the plan kernel lists the pairs, heaviest sequences first.  Warp roles:
-//   warp 0      TMA producer: Q_A, Q_B, then K_j and V_j tiles into a 4-stage ring
-//               (one 3-D tensor-map box per cache block piece; a 128-key tile spans
-//               128 / block_size blocks when the block size is below 128);
+//   warp 0      TMA producer: Q_A, K_0, Q_B, V_0, then K_j and V_j tiles into a 4-stage
+//               ring (one 3-D tensor-map box per cache block piece; a 128-key tile spans
+//               128 / block_size blocks when the block size is below 128).  Q_B's buffer
+//               frees last (tile B has the most key tiles), so it is loaded after K_0;
+//               the MMA issuer likewise starts S_A0 before waiting for Q_B;
 //   warp 1      allocates all 512 TMEM columns; one lane issues the MMAs in the order
 //                 S_A0 S_B0 | O_A += P_A0 V_0, S_A1, O_B += P_B0 V_0, S_B1 | ...
 //               where S = Q K_j^T is SS (both operands K-major in shared memory) and
@@ -464,13 +466,12 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             const int bt_seq = PREFIX ? __ldg(p.members + ta.q0) : ta.seq;   // a member's table
             const int32_t* bt = p.block_tables + (size_t)bt_seq * p.max_blocks;
             int cur_blk = load_pieces(bt, ta.kbeg, ta.lk, 0);
-            for (int x = 0; x < 2 && ok; ++x) {
+            // Q tile x of this unit (its buffer frees after the last S of the previous unit's
+            // tile x)
+            auto load_q = [&](int x) -> bool {
                 const TileInfo& t = x ? tb : ta;
-                if (!t.valid) continue;
-                if (!mbar_wait(bars + L::B_QEMPTY + x, (qloads[x] & 1) ^ 1, abort_flag, p.err)) {
-                    ok = false;
-                    break;
-                }
+                if (!t.valid) return true;
+                if (!mbar_wait(bars + L::B_QEMPTY + x, (qloads[x] & 1) ^ 1, abort_flag, p.err)) return false;
                 uint8_t* qdst = smem + L::Q_OFF + x * L::TILE_BYTES;
                 if constexpr (PREFIX) {
                     // gather the members' query rows into the swizzled Q tile with 16-byte
@@ -511,35 +512,42 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                     }
                 }
                 ++qloads[x];
-            }
+                return true;
+            };
+            // K (kv = 0) or V tile j, whose block pieces lane c holds in blk_lane
+            auto load_kv = [&](int kv, int j, int blk_lane) -> bool {
+                const int slot = fill % kStages;
+                if (!mbar_wait(bars + L::B_KVEMPTY + slot, ((fill / kStages) & 1) ^ 1, abort_flag, p.err))
+                    return false;
+                const uint32_t valid_mask = __ballot_sync(0xffffffffu, blk_lane >= 0);
+                const uint32_t bytes = (uint32_t)__popc(valid_mask) * (uint32_t)(piece * 128 * L::REGIONS);
+                uint8_t* dst = smem + L::STAGE_OFF + slot * L::TILE_BYTES;
+                const CUtensorMap* map = kv ? &v_map : &k_map;
+                if (lane == 0) mbar_arrive_expect_tx(bars + L::B_KVFULL + slot, bytes);
+                for (uint32_t m = valid_mask; m != 0; m &= m - 1) {
+                    const int c = __ffs(m) - 1;
+                    const int blk = __shfl_sync(0xffffffffu, blk_lane, c);
+                    if (lane == 0) {
+                        const int kc = ta.kbeg + j * kKV + c * piece;
+                        const int z = blk * p.block_size + (kc & (p.block_size - 1));
+                        for (int r = 0; r < L::REGIONS; ++r)
+                            tma_load_3d(dst + r * L::REGION_BYTES + c * piece * 128, map, bars + L::B_KVFULL + slot,
+                                        r * 64, ta.hk, z);
+                    }
+                }
+                last_fill[slot] = (int)fill;
+                ++fill;
+                return true;
+            };
+            // Q_A, K_0, Q_B, V_0, then K_j, V_j: tile B's Q buffer frees last (B has the most
+            // key tiles), so K_0 and tile A's first S do not wait for it
+            ok = load_q(0);
+            if (ok && nkv > 0) ok = load_kv(0, 0, cur_blk);
+            if (ok) ok = load_q(1);
             for (int j = 0; j < nkv && ok; ++j) {
                 const int nxt_blk = j + 1 < nkv ? load_pieces(bt, ta.kbeg, ta.lk, j + 1) : -1;
-                const int key0 = j * kKV;
-                const uint32_t valid_mask = __ballot_sync(0xffffffffu, cur_blk >= 0);
-                const uint32_t bytes = (uint32_t)__popc(valid_mask) * (uint32_t)(piece * 128 * L::REGIONS);
-                for (int kv = 0; kv < 2; ++kv) {
-                    const int slot = fill % kStages;
-                    if (!mbar_wait(bars + L::B_KVEMPTY + slot, ((fill / kStages) & 1) ^ 1, abort_flag, p.err)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t* dst = smem + L::STAGE_OFF + slot * L::TILE_BYTES;
-                    const CUtensorMap* map = kv ? &v_map : &k_map;
-                    if (lane == 0) mbar_arrive_expect_tx(bars + L::B_KVFULL + slot, bytes);
-                    for (uint32_t m = valid_mask; m != 0; m &= m - 1) {
-                        const int c = __ffs(m) - 1;
-                        const int blk = __shfl_sync(0xffffffffu, cur_blk, c);
-                        if (lane == 0) {
-                            const int kc = ta.kbeg + key0 + c * piece;
-                            const int z = blk * p.block_size + (kc & (p.block_size - 1));
-                            for (int r = 0; r < L::REGIONS; ++r)
-                                tma_load_3d(dst + r * L::REGION_BYTES + c * piece * 128, map,
-                                            bars + L::B_KVFULL + slot, r * 64, ta.hk, z);
-                        }
-                    }
-                    last_fill[slot] = (int)fill;
-                    ++fill;
-                }
+                if (j > 0) ok = load_kv(0, j, cur_blk);
+                if (ok) ok = load_kv(1, j, cur_blk);
                 cur_blk = nxt_blk;
             }
         }
@@ -602,21 +610,24 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             const int nk[2] = {ta.nkv, tb.nkv};
             const bool val[2] = {ta.valid, tb.valid};
             const int nkv = max(nk[0], nk[1]);
-            for (int x = 0; x < 2 && ok; ++x)
-                if (val[x] && !mbar_wait(bars + L::B_QFULL + x, quse[x] & 1, abort_flag, p.err)) ok = false;
-            if (!ok) break;
-            if (nkv > 0) {
-                const int kslot = fbase % kStages;
-                if (!mbar_wait(bars + L::B_KVFULL + kslot, (fbase / kStages) & 1, abort_flag, p.err)) break;
-            }
-            tc_fence_after();
-            if (lane == 0) {
-                for (int x = 0; x < 2; ++x) {
-                    if (nk[x] > 0) issue_qk(x, fbase % kStages);
-                    if (val[x] && nk[x] <= 1) umma_commit(bars + L::B_QEMPTY + x);
+            // S of key tile 0: tile A as soon as Q_A and K_0 are in, then tile B
+            if (nkv > 0 && !mbar_wait(bars + L::B_KVFULL + fbase % kStages, (fbase / kStages) & 1, abort_flag, p.err))
+                break;
+            for (int x = 0; x < 2 && ok; ++x) {
+                if (!val[x]) continue;
+                if (!mbar_wait(bars + L::B_QFULL + x, quse[x] & 1, abort_flag, p.err)) {
+                    ok = false;
+                    break;
                 }
-                if (nkv > 0) umma_commit(bars + L::B_KVEMPTY + fbase % kStages);
+                tc_fence_after();
+                if (lane == 0) {
+                    if (nk[x] > 0) issue_qk(x, fbase % kStages);
+                    if (nk[x] <= 1) umma_commit(bars + L::B_QEMPTY + x);
+                }
+                __syncwarp();
             }
+            if (!ok) break;
+            if (nkv > 0 && lane == 0) umma_commit(bars + L::B_KVEMPTY + fbase % kStages);
             __syncwarp();
             for (int j = 0; j < nkv && ok; ++j) {
                 const uint32_t fv = fbase + 2 * (uint32_t)j + 1, fk = fv + 1;
