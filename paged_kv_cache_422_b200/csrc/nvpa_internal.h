@@ -75,6 +75,7 @@ struct DecodePrefixArgs {
     int32_t* err_flag;
     const int4* tiles;           // (group, query tile A, query tile B or -1, partition)
     const int32_t* ntiles;
+    int32_t* unit_counter;       // zeroed by the plan; the kernel claims work units from it
     const int32_t* members;
     const int32_t* group_start;
     const int32_t* group_len;

@@ -161,7 +161,8 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const AttnParams p) {
 //   private partitions npc .. npc+nsp-1 keys [prefix + s * chunk, ...), worker items;
 // and the combine merges all npc + nsp partials.  Sequences outside a group get the plain
 // decode plan's items.  Counters in the workspace: [0] next item, [1] items, [2] groups,
-// [3] members, [4] prefix work units (pairs of query tiles of one group and partition).
+// [3] members, [4] prefix work units (pairs of query tiles of one group and partition),
+// [5] the prefix kernel's unit counter.
 constexpr int kSharedTable = 2 * kSharedMaxBatch;   // a power of two above the batch
 
 __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& total) {
@@ -354,6 +355,7 @@ __global__ void __launch_bounds__(1024) decode_plan_shared_kernel(const AttnPara
         p.counter[2] = ngroups;
         p.counter[3] = nmembers;
         p.counter[4] = s_ntiles;
+        p.counter[5] = 0;   // the prefix kernel's unit counter
     }
 }
 
@@ -885,6 +887,7 @@ nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream) {
         a.err_flag = c.err_flag;
         a.tiles = p.ptiles;
         a.ntiles = p.counter + 4;
+        a.unit_counter = p.counter + 5;
         a.members = p.members;
         a.group_start = p.group_start;
         a.group_len = p.group_len;

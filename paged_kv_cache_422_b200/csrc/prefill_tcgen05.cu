@@ -67,6 +67,8 @@ static_assert(4 * kSmallRegs + 8 * kSoftmaxRegs == 12 * kLaunchRegs, "register s
 static_assert((kSmallRegs + 2 * kSoftmaxRegs) * 32 <= 16384, "sub-partition registers");
 constexpr int kTmemCols = 512;   // 2 tiles x (S/P 128 + O up to 128)
 constexpr int kMinTokensPerTile = 16;   // 128 rows / at most 8 packed heads
+constexpr int kUnitRing = 4;            // claimed unit indices handed from the producer to the others
+constexpr int kUnitReaders = 1 + 8;     // MMA warp + the 8 softmax warps
 
 // Bit k set for the first n of 32 columns (n clamped to [0, 32]).
 __device__ __forceinline__ uint32_t visible_mask(int n) {
@@ -163,6 +165,7 @@ struct PrefillParams {
     int32_t* err;
     const int4* tiles;           // plan: (sequence, query tile A, query tile B or -1, key partition)
     const int32_t* ntiles;       // plan: number of entries
+    int32_t* unit_counter;       // next unit to claim (reset by the plan)
     // shared-prefix decode mode: "sequences" are prefix groups whose "queries" are the
     // members' decode query rows; results go to each member's prefix partition slot
     const uint16_t* q_rows;      // decode q [batch, Hq, D]
@@ -194,9 +197,10 @@ struct Layout {
     static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KVFULL = 4, B_KVEMPTY = B_KVFULL + kStages;
     static constexpr int B_SFULL = B_KVEMPTY + kStages, B_PFULL = B_SFULL + 2, B_ODONE = B_PFULL + 2;
     static constexpr int B_OFINAL = B_ODONE + 2, B_OFREE = B_OFINAL + 2, B_DRAIN = B_OFREE + 2;
-    static constexpr int NBARS = B_DRAIN + 1;
-    static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;     // tmem base, abort flag
-    static constexpr int BYTES = MISC_OFF + 16;
+    static constexpr int B_UFULL = B_DRAIN + 1, B_UEMPTY = B_UFULL + kUnitRing;
+    static constexpr int NBARS = B_UEMPTY + kUnitRing;
+    static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;     // tmem base, abort flag, unit ring
+    static constexpr int BYTES = MISC_OFF + 16 + 4 * kUnitRing;
     static constexpr int ALLOC = BYTES + 1024;               // room to align the base to 1024
 };
 
@@ -370,7 +374,10 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const PrefillParams 
         __syncthreads();
         if (tid == 0) written = extra_base;
     }
-    if (tid == 0) *ntiles = written;
+    if (tid == 0) {
+        *ntiles = written;
+        ntiles[1] = 0;   // the attention kernel's unit counter
+    }
 }
 
 // ------------------------------------------------------------------------------------
@@ -389,6 +396,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+    volatile int* unit_ring = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 16);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if constexpr (PREFIX) {
@@ -413,6 +421,10 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             mbar_init(bars + L::B_KVEMPTY + s, 1);
         }
         mbar_init(bars + L::B_DRAIN, 1);
+        for (int i = 0; i < kUnitRing; ++i) {
+            mbar_init(bars + L::B_UFULL + i, 1);
+            mbar_init(bars + L::B_UEMPTY + i, kUnitReaders);
+        }
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&q_map);
@@ -429,6 +441,18 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
     const uint32_t tmem = *tmem_slot;
 
     const int total = __ldcg(p.ntiles) * p.hgroups;
+    // Units are claimed dynamically (longest first, as the plan orders them): the producer
+    // claims the next one with an atomic and hands its index to the MMA and softmax warps
+    // through a small ring in shared memory; -1 ends the loop.  claim(n) returns the n-th
+    // unit of this CTA, -1 at the end, -2 if a wait timed out.
+    auto claim = [&](int n) -> int {
+        const int slot = n % kUnitRing;
+        if (!mbar_wait(bars + L::B_UFULL + slot, (n / kUnitRing) & 1, abort_flag, p.err)) return -2;
+        const int idx = unit_ring[slot];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + L::B_UEMPTY + slot);
+        return idx;
+    };
 
     if (warp < 4) {
       // warpgroup 0: producer, MMA issuer and two idle warps, with few registers
@@ -457,7 +481,18 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             return blk;
         };
         bool ok = true;
-        for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
+        for (int n = 0; ok; ++n) {
+            const int slot = n % kUnitRing;
+            if (!mbar_wait(bars + L::B_UEMPTY + slot, ((n / kUnitRing) & 1) ^ 1, abort_flag, p.err)) break;
+            int idx = 0;
+            if (lane == 0) {
+                idx = atomicAdd(p.unit_counter, 1);
+                if (idx >= total) idx = -1;
+                unit_ring[slot] = idx;
+                mbar_arrive(bars + L::B_UFULL + slot);
+            }
+            idx = __shfl_sync(0xffffffffu, idx, 0);
+            if (idx < 0) break;
             const int4 e = __ldg(p.tiles + idx / p.hgroups);
             const int hg = idx % p.hgroups;
             const TileInfo ta = tile_info<PREFIX>(p, e, hg, false);
@@ -602,7 +637,9 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             }
             umma_commit(bars + L::B_ODONE + x);
         };
-        for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
+        for (int n = 0; ok; ++n) {
+            const int idx = claim(n);
+            if (idx < 0) break;
             const int4 e = __ldg(p.tiles + idx / p.hgroups);
             const int hg = idx % p.hgroups;
             const TileInfo ta = tile_info<PREFIX>(p, e, hg, false);
@@ -719,7 +756,9 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
         uint32_t s_use = 0;
         int tcount = 0;
         uint32_t pv_before = 0;                       // PVs issued for this tile slot before
-        for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
+        for (int n = 0;; ++n) {
+            const int idx = claim(n);
+            if (idx < 0) break;
             const TileInfo t = tile_info<PREFIX>(p, __ldg(p.tiles + idx / p.hgroups), idx % p.hgroups, x == 1);
             if (t.nkv == 0) continue;
             const int pos = t.lk - t.lq + t.tok0 + rtok;           // absolute position of this row
@@ -937,6 +976,7 @@ cudaError_t launch_decode_prefix_tcgen05(const DecodePrefixArgs& a, cudaStream_t
     p.err = a.err_flag;
     p.tiles = a.tiles;
     p.ntiles = a.ntiles;
+    p.unit_counter = a.unit_counter;
     p.q_rows = static_cast<const uint16_t*>(a.q);
     p.members = a.members;
     p.group_start = a.group_start;
@@ -999,6 +1039,7 @@ nvpa_status_t run_varlen_prefill_tcgen05(const PrefillCall& c, void* workspace, 
     p.lse_out = c.lse_out;
     p.err = c.err_flag;
     p.ntiles = reinterpret_cast<int32_t*>(ws);
+    p.unit_counter = reinterpret_cast<int32_t*>(ws) + 1;
     p.tiles = reinterpret_cast<const int4*>(ws + 256);
     p.batch = c.batch;
     p.total_q = c.total_q;
