@@ -183,6 +183,13 @@ DECODE_SOURCES = ["paged_kv_cache_422_b200/csrc/paged_attention.cu",
                   "paged_kv_cache_422_b200/csrc/common.cuh"]
 
 
+# sources of the tcgen05 attention kernel, the dominant kernel of a prefill step
+PREFILL_SOURCES = ["paged_kv_cache_422_b200/csrc/prefill_tcgen05.cu",
+                   "paged_kv_cache_422_b200/csrc/sm100.cuh",
+                   "paged_kv_cache_422_b200/csrc/attn_warp.cuh",
+                   "paged_kv_cache_422_b200/csrc/common.cuh"]
+
+
 def source_sha(files) -> str:
     digest = hashlib.sha256()
     for f in files:
@@ -525,7 +532,9 @@ def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
                     l2="not flushed: K/V of the step (about 140 MB) is near the 126 MB L2"),
         roofline=dict(bound="tensor", kernel="varlen_prefill_attention (plan + tcgen05 kernel)",
                       achieved=attn_tflops, peak=peaks["bf16_tflops"], unit="TFLOP/s",
-                      frac=attn_tflops / peaks["bf16_tflops"], traffic=None,
+                      frac=attn_tflops / peaks["bf16_tflops"],
+                      traffic=(profile_traffic("prefill_tcgen05_varlen_b32", PREFILL_SOURCES)
+                               if args.workload == "prefill_varlen_prefix_hits_b32" else None),
                       peak_source=peaks["source"] + " (MEASURED_PEAKS.json bf16_tflops, burst)"),
         gpu_launches=int(launches), clocks=clocks.summary())
     if rank == 0:

@@ -440,7 +440,19 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    const int total = __ldcg(p.ntiles) * p.hgroups;
+    // Work units: every plan entry for every head group.  In the shared-prefix mode the
+    // work is small (a few groups' prefixes) and latency-bound, so each pair entry is
+    // split into two single-tile units for twice the parallelism.
+    const int total = __ldcg(p.ntiles) * p.hgroups * (PREFIX ? 2 : 1);
+    auto unit_of = [&](int idx, int4& e, int& hg) {
+        hg = idx % p.hgroups;
+        if constexpr (PREFIX) {
+            const int4 pe = __ldg(p.tiles + idx / (2 * p.hgroups));
+            e = make_int4(pe.x, ((idx / p.hgroups) & 1) ? pe.z : pe.y, -1, pe.w);
+        } else {
+            e = __ldg(p.tiles + idx / p.hgroups);
+        }
+    };
     // Units are claimed dynamically (longest first, as the plan orders them): the producer
     // claims the next one with an atomic and hands its index to the MMA and softmax warps
     // through a small ring in shared memory; -1 ends the loop.  claim(n) returns the n-th
@@ -493,8 +505,9 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             }
             idx = __shfl_sync(0xffffffffu, idx, 0);
             if (idx < 0) break;
-            const int4 e = __ldg(p.tiles + idx / p.hgroups);
-            const int hg = idx % p.hgroups;
+            int4 e;
+            int hg;
+            unit_of(idx, e, hg);
             const TileInfo ta = tile_info<PREFIX>(p, e, hg, false);
             const TileInfo tb = tile_info<PREFIX>(p, e, hg, true);
             const int nkv = max(ta.nkv, tb.nkv);
@@ -640,8 +653,9 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
         for (int n = 0; ok; ++n) {
             const int idx = claim(n);
             if (idx < 0) break;
-            const int4 e = __ldg(p.tiles + idx / p.hgroups);
-            const int hg = idx % p.hgroups;
+            int4 e;
+            int hg;
+            unit_of(idx, e, hg);
             const TileInfo ta = tile_info<PREFIX>(p, e, hg, false);
             const TileInfo tb = tile_info<PREFIX>(p, e, hg, true);
             const int nk[2] = {ta.nkv, tb.nkv};
@@ -759,7 +773,10 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
         for (int n = 0;; ++n) {
             const int idx = claim(n);
             if (idx < 0) break;
-            const TileInfo t = tile_info<PREFIX>(p, __ldg(p.tiles + idx / p.hgroups), idx % p.hgroups, x == 1);
+            int4 e;
+            int hg;
+            unit_of(idx, e, hg);
+            const TileInfo t = tile_info<PREFIX>(p, e, hg, x == 1);
             if (t.nkv == 0) continue;
             const int pos = t.lk - t.lq + t.tok0 + rtok;           // absolute position of this row
             const int lim = (!PREFIX && p.causal) ? min(t.lk, pos + 1) : t.lk;  // keys 0 .. lim-1 visible
@@ -998,7 +1015,7 @@ cudaError_t launch_decode_prefix_tcgen05(const DecodePrefixArgs& a, cudaStream_t
     p.block_size = a.block_size;
     p.block_shift = __builtin_ctz((unsigned)a.block_size);
     p.scale_log2 = a.scale * kLog2e;
-    const long long units = std::max(1LL, a.max_entries) * p.hgroups;
+    const long long units = std::max(1LL, a.max_entries) * p.hgroups * 2;   // single-tile units
     const long long cap = a.max_ctas > 0 ? a.max_ctas : (long long)device_sm_count();
     const int grid = (int)std::max(1LL, std::min<long long>(cap, units));
     // the query map is not read in this mode (rows are gathered); any valid map will do
