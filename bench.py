@@ -179,6 +179,7 @@ def profile_traffic(kernel_tag: str, source_files) -> float | None:
 
 # sources of the split-KV worker, the dominant kernel of a decode step
 DECODE_SOURCES = ["paged_kv_cache_422_b200/csrc/paged_attention.cu",
+                  "paged_kv_cache_422_b200/csrc/decode_params.cuh",
                   "paged_kv_cache_422_b200/csrc/attn_warp.cuh",
                   "paged_kv_cache_422_b200/csrc/common.cuh"]
 

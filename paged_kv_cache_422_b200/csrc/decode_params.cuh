@@ -1,0 +1,80 @@
+// Parameters and launch helpers shared by the paged decode kernels (plan, shared-prefix
+// plan, split-KV worker, combine).
+#pragma once
+
+#include <climits>
+
+#include "attn_warp.cuh"
+#include "nvpa_internal.h"
+
+namespace nvpa {
+
+#ifndef NVPA_DECODE_STAGES
+#define NVPA_DECODE_STAGES 2
+#endif
+
+constexpr int kAttnWarps = 4;
+constexpr int kAttnStages = NVPA_DECODE_STAGES;
+constexpr int kSharedMaxBatch = 2048;   // larger batches are decoded without prefix groups
+constexpr int kDefaultMinGroup = 8;
+
+struct AttnParams {
+    const uint16_t* q;
+    const uint16_t* k_cache;
+    const uint16_t* v_cache;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    // fused decode step: sequence b's newest key/value (position context_lens[b]-1) is read
+    // from k_new/v_new row b instead of the cache and written to slot_mapping[b]
+    const uint16_t* k_new;
+    const uint16_t* v_new;
+    long long k_new_stride, v_new_stride;   // elements between rows of k_new / v_new
+    const int32_t* slot_mapping;
+    long long capacity;                     // num_blocks * block_size
+    int fused;
+    uint16_t* k_cache_w;
+    uint16_t* v_cache_w;
+    uint16_t* out;
+    float* out_f32;                // partial mode: fp32 normalised output instead of bf16 `out`
+    float* lse_out;
+    float* o_part;
+    float* lse_part;
+    int4* items;
+    int32_t* nsplit;
+    int32_t* counter;              // [0] next item, [1] number of items
+    int32_t* err;
+    int batch, hq, hkv, group;
+    int max_blocks, num_blocks, block_size, block_shift;
+    int max_ctx;                   // host-side bound of context_lens
+    int chunk, s_max;              // keys per partition, partitions of the longest context
+    float scale_log2;
+    // shared-prefix plan outputs (decode_plan_shared_kernel)
+    int4* ptiles;                  // (group, query tile A, query tile B or -1, prefix partition)
+    int32_t* members;              // grouped member lists
+    int32_t* group_start;          // [groups + 1]
+    int32_t* group_len;            // [groups] prefix tokens
+    int min_members, pchunk, ptq;  // smallest group, prefix keys per partition, members per tile
+};
+
+template <int D, int GMAX>
+struct AttnStage {
+    static constexpr int KV_BYTES = kTileKeys * D * 2;
+    static constexpr int Q_BYTES = GMAX * D * 2;
+    static constexpr int BYTES = 2 * KV_BYTES + Q_BYTES + 32;   // + two int4 of metadata
+};
+
+// Programmatic dependent launch: wait for the preceding kernel's results / let the next
+// kernel's CTAs start launching.  Both are no-ops for a normal launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+
+constexpr int kSharedTable = 2 * kSharedMaxBatch;   // buckets of the shared-prefix plan (a power of two)
+constexpr size_t kSharedPlanSmem = sizeof(int) * (6 * (size_t)kSharedTable + 2 * (size_t)kSharedMaxBatch);
+
+// Enqueue the shared-prefix plan (one CTA) on `stream`.
+cudaError_t launch_decode_plan_shared(const AttnParams& p, cudaStream_t stream);
+
+}  // namespace nvpa
