@@ -13,8 +13,8 @@
 // last token's position (bottom-right alignment: suffix token r is at position
 // Lk - Lq + r).
 //
-// Work unit: a PAIR of query tiles of the same sequence and KV head (A = tile q, B = tile
-// q + 1, the one with more key tiles; B may be absent).  Both read the same K/V tiles, so
+// Work unit: a PAIR of query tiles of the same sequence and KV head (A = tile 2w, B = tile
+// 2w + 1, which has at least as many key tiles; B may be absent).  Both read the same K/V tiles, so
 // each tile is fetched once for 256 query rows, and the two tiles' MMAs and softmaxes
 // interleave: while one tile's softmax runs, the tensor core computes the other tile's
 // P V and its next S.  One CTA per SM (persistent; CTA c takes units c, c + grid, ...);
@@ -258,12 +258,16 @@ constexpr int kPlanMaxRanked = 2048;   // batches up to this size are ordered by
 // all their query tiles) first and, inside a sequence, the pairs with the most key tiles
 // first.  CTAs that run at the same time then mostly read the same sequences' keys and
 // values, which L2 serves after the first fetch, and the longest work starts first.  A
-// sequence with cnt query tiles gives the pairs (cnt-2, cnt-1), (cnt-4, cnt-3), ... and,
-// for odd cnt, the single tile 0.
+// sequence with cnt query tiles gives the pairs (2w, 2w+1) counted from its first tile,
+// last pair first; for odd cnt the last tile stands alone.  Counting from the first tile
+// aligns a pair with the 128-key tiles when 2 * tokens per tile = 128 and the cached
+// prefix is a whole number of 128-key tiles (block sizes of 128 and 256): both tiles of
+// a pair then end in the same key tile and finish their key loops together.
 __device__ __forceinline__ void write_pairs(int4* tiles, int off, int seq, int cnt) {
-    for (int u = 0; 2 * u < cnt; ++u) {
-        const int b = cnt - 1 - 2 * u;
-        tiles[off + u] = b >= 1 ? make_int4(seq, b - 1, b, 0) : make_int4(seq, 0, -1, 0);
+    const int npairs = (cnt + 1) / 2;
+    for (int u = 0; u < npairs; ++u) {
+        const int w = npairs - 1 - u;
+        tiles[off + u] = make_int4(seq, 2 * w, 2 * w + 1 < cnt ? 2 * w + 1 : -1, 0);
     }
 }
 
