@@ -51,6 +51,8 @@ CASES = [
     ([64, 64], [4, 0], 6, 2, 128, 16),          # first sequence fully cached: Lq = 0
     ([200, 31, 77], [3, 0, 2], 12, 4, 64, 32),
     ([700], [1], 8, 1, 128, 128),
+    ([450, 97], [2, 0], 8, 2, 128, 64),           # group 4: four heads per tile row block
+    ([1500, 5], [5, 0], 16, 8, 128, 128),         # many query-tile pairs, prefix of 640 keys
 ]
 
 
