@@ -74,7 +74,28 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 constexpr int kSharedTable = 2 * kSharedMaxBatch;   // buckets of the shared-prefix plan (a power of two)
 constexpr size_t kSharedPlanSmem = sizeof(int) * (6 * (size_t)kSharedTable + 2 * (size_t)kSharedMaxBatch);
 
+// Launch with programmatic stream serialisation: the kernel may start while its
+// predecessor finishes and synchronises with it through griddepcontrol.wait.
+template <typename Kernel>
+cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       const AttnParams& p) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 // Enqueue the shared-prefix plan (one CTA) on `stream`.
 cudaError_t launch_decode_plan_shared(const AttnParams& p, cudaStream_t stream);
+// Enqueue the split-KV combine (grid CTAs of 8 warps, one warp per sequence and query
+// head), as a programmatic dependent of the worker.
+cudaError_t launch_decode_combine(const AttnParams& p, int head_dim, int grid, cudaStream_t stream);
 
 }  // namespace nvpa

@@ -299,104 +299,9 @@ paged_attention_kernel(const AttnParams p) {
 }
 
 // ------------------------------------------------------------------------------------
-// combine: merge the partitions of every (sequence, query head) that has more than one
-// ------------------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(256) decode_combine_kernel(const AttnParams p) {
-    constexpr int DPL = D / 32;   // output dims per lane
-    pdl_wait();
-    const int w = blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (w >= p.batch * p.hq) return;
-    const int b = w / p.hq;
-    const int ns = __ldcg(p.nsplit + b);
-    if (ns <= 1) return;
-    const float* lp = p.lse_part + (size_t)w * p.s_max;
-    const float* op = p.o_part + (size_t)w * p.s_max * D + lane * DPL;
-    float mx = -INFINITY;
-    for (int s = lane; s < ns; s += 32) mx = fmaxf(mx, __ldcg(lp + s));
-    mx = warp_max(mx);
-    float acc[DPL];
-#pragma unroll
-    for (int k = 0; k < DPL; ++k) acc[k] = 0.f;
-    float tot = 0.f;
-    if (mx > -INFINITY) {
-        for (int s0 = 0; s0 < ns; s0 += 32) {
-            const float wl = (s0 + lane < ns) ? fast_exp2((__ldcg(lp + s0 + lane) - mx) * kLog2e) : 0.f;
-            tot += wl;
-            const int n = min(32, ns - s0);
-            int j = 0;
-            for (; j + 4 <= n; j += 4) {   // four independent loads in flight
-                float ws[4];
-                float v[4][DPL];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    ws[u] = __shfl_sync(0xffffffffu, wl, j + u);
-                    const float* src = op + (size_t)(s0 + j + u) * D;
-                    if constexpr (DPL == 4) {
-                        const float4 t = __ldcg(reinterpret_cast<const float4*>(src));
-                        v[u][0] = t.x; v[u][1] = t.y; v[u][2] = t.z; v[u][3] = t.w;
-                    } else {
-                        const float2 t = __ldcg(reinterpret_cast<const float2*>(src));
-                        v[u][0] = t.x; v[u][1] = t.y;
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-#pragma unroll
-                    for (int k = 0; k < DPL; ++k) acc[k] = fmaf(ws[u], v[u][k], acc[k]);
-            }
-            for (; j < n; ++j) {
-                const float ws = __shfl_sync(0xffffffffu, wl, j);
-                const float* src = op + (size_t)(s0 + j) * D;
-#pragma unroll
-                for (int k = 0; k < DPL; ++k) acc[k] = fmaf(ws, __ldcg(src + k), acc[k]);
-            }
-        }
-        tot = warp_sum(tot);
-    }
-    const float inv = tot > 0.f ? 1.f / tot : 0.f;
-    if (p.out_f32 != nullptr) {
-        float* dst = p.out_f32 + (size_t)w * D + lane * DPL;
-#pragma unroll
-        for (int k = 0; k < DPL; ++k) dst[k] = acc[k] * inv;
-        if (lane == 0 && p.lse_out != nullptr) p.lse_out[w] = tot > 0.f ? mx + __logf(tot) : -INFINITY;
-        return;
-    }
-    uint16_t* dst = p.out + (size_t)w * D + lane * DPL;
-    if constexpr (DPL == 4) {
-        uint2 v;
-        v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-        v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-        *reinterpret_cast<uint2*>(dst) = v;
-    } else {
-        *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-    }
-    if (lane == 0 && p.lse_out != nullptr) p.lse_out[w] = tot > 0.f ? mx + __logf(tot) : -INFINITY;
-}
-
-// ------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------
 namespace {
-
-// Launch with programmatic stream serialisation: the kernel may start while its
-// predecessor finishes and synchronises with it through griddepcontrol.wait.
-template <typename Kernel>
-cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                       const AttnParams& p) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, p);
-}
 
 template <int D, int GMAX>
 int worker_ctas_per_sm() {
@@ -627,8 +532,7 @@ nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream) {
     if (s_max > 1) {
         const long long warps = (long long)c.batch * c.hq;
         const int grid = (int)((warps + 7) / 8);
-        e = c.head_dim == 128 ? launch_pdl(decode_combine_kernel<128>, dim3(grid), dim3(256), 0, stream, p)
-                              : launch_pdl(decode_combine_kernel<64>, dim3(grid), dim3(256), 0, stream, p);
+        e = launch_decode_combine(p, c.head_dim, grid, stream);
         if (e != cudaSuccess) return cuda_failure(e, "decode combine launch");
         count_launches(1);
     }
