@@ -19,7 +19,7 @@
 // interleave: while one tile's softmax runs, the tensor core computes the other tile's
 // P V and its next S.  One CTA per SM (persistent; CTA c takes units c, c + grid, ...);
 // the plan kernel lists the pairs, heaviest sequences first.  Warp roles:
-//   warp 0      TMA producer: Q_A, K_0, Q_B, V_0, then K_j and V_j tiles into a 4-stage
+//   warp 0      TMA producer: Q_A, K_0, Q_B, V_0, then K_j and V_j tiles into a 5-stage
 //               ring (one 3-D tensor-map box per cache block piece; a 128-key tile spans
 //               128 / block_size blocks when the block size is below 128).  Q_B's buffer
 //               frees last (tile B has the most key tiles), so it is loaded after K_0;
@@ -40,6 +40,7 @@
 // in the last key tile are zeroed in shared memory before their MMAs, so a 0 weight
 // never meets a NaN.
 #include <algorithm>
+#include <climits>
 #include <mutex>
 
 #include "attn_warp.cuh"
@@ -54,7 +55,11 @@ namespace {
 
 constexpr int kQ = 128;          // query rows per tile (MMA M): tokens x packed heads
 constexpr int kKV = 128;         // keys per tile (MMA N of QK^T, K of PV)
-constexpr int kStages = 4;       // K/V ring stages, each one K or one V tile
+// K/V ring stages, each one K or one V tile.  A tile takes about 2 us from the TMA issue to
+// its arrival under load, about one key-tile period of a pair, so the producer must run
+// more than a period ahead: with 5 stages V_{j+2} is issued once K_j is consumed.  Five
+// 32 KB stages and the two Q tiles fill the 227 KB of shared memory a CTA may have.
+constexpr int kStages = 5;
 constexpr int kWarps = 12;       // producer, MMA, 2 idle, 2 x 4 softmax
 constexpr int kThreads = kWarps * 32;
 // Register split (setmaxnreg acts on whole warpgroups): the launch gives every thread
@@ -87,73 +92,75 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     return d;
 }
 
-__device__ __forceinline__ float min3(float a, float b, float c) {
-    float d;
-    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
+// The softmax of one S row (one thread per row, the whole 128-column row in registers) is a
+// single code path for every tile and either sign of the scale, kept small on purpose: the
+// warps that issue the MMAs and the copies share each SM sub-partition's instruction
+// cache with two softmax warps, and the fully unrolled row loops are most of the kernel's
+// code.
 
-// Max (MAX) or min of the visible raw scores of one 128-column S row; with MASK only the
-// columns below lim - key0 count (masked ones become -inf / +inf by bit mask).  Two
-// independent accumulators, two new scores per three-input instruction.
-template <bool MAX, bool MASK>
-__device__ __forceinline__ float row_extreme(const uint32_t (&sv)[kKV], int key0, int lim) {
-    const float fill = MAX ? -INFINITY : INFINITY;
-    float e0 = fill, e1 = fill;
+// x = s * scale (log2 units) in place, two scores per packed multiply.
+__device__ __forceinline__ void scale_row(uint32_t (&sv)[kKV], float sc) {
+    const uint64_t sc2 = f2_pack(sc, sc);
 #pragma unroll
-    for (int c = 0; c < kKV / 32; ++c) {
-        const uint32_t vm = MASK ? visible_mask(lim - key0 - c * 32) : 0xffffffffu;
-#pragma unroll
-        for (int k = 0; k < 32; k += 4) {
-            float x0 = __uint_as_float(sv[c * 32 + k]), x1 = __uint_as_float(sv[c * 32 + k + 1]);
-            float x2 = __uint_as_float(sv[c * 32 + k + 2]), x3 = __uint_as_float(sv[c * 32 + k + 3]);
-            if (MASK) {
-                x0 = keep_or(sv[c * 32 + k], vm, k, fill);
-                x1 = keep_or(sv[c * 32 + k + 1], vm, k + 1, fill);
-                x2 = keep_or(sv[c * 32 + k + 2], vm, k + 2, fill);
-                x3 = keep_or(sv[c * 32 + k + 3], vm, k + 3, fill);
-            }
-            e0 = MAX ? max3(e0, x0, x1) : min3(e0, x0, x1);
-            e1 = MAX ? max3(e1, x2, x3) : min3(e1, x2, x3);
-        }
+    for (int k = 0; k < kKV; k += 2) {
+        float a, b;
+        f2_unpack(f2_mul(f2_pack(__uint_as_float(sv[k]), __uint_as_float(sv[k + 1])), sc2), a, b);
+        sv[k] = __float_as_uint(a);
+        sv[k + 1] = __float_as_uint(b);
     }
-    return MAX ? fmaxf(e0, e1) : fminf(e0, e1);
 }
 
-// P = exp2(s * sce + nme) of one S row, packed to bf16 pairs and written over the first
-// kKV/2 TMEM columns of the row (32 S columns become 16 P columns, each chunk's P landing
-// in columns already read); returns the row sum of the fp32 values.  With MASK, columns
-// at or past lim - key0 get 0 by bit mask.
-template <bool MASK>
-__device__ __forceinline__ float exp_row(const uint32_t (&sv)[kKV], uint32_t s_col, float sce, float nme,
-                                         int key0, int lim) {
-    float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+// Columns at or past lim - key0 (keys the row does not see, including rows past the
+// sequence) become -inf by bit mask, whatever they held.
+__device__ __forceinline__ void mask_row(uint32_t (&sv)[kKV], int key0, int lim) {
 #pragma unroll
     for (int c = 0; c < kKV / 32; ++c) {
-        const uint32_t vm = MASK ? visible_mask(lim - key0 - c * 32) : 0xffffffffu;
+        const uint32_t vm = visible_mask(lim - key0 - c * 32);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) sv[c * 32 + k] = __float_as_uint(keep_or(sv[c * 32 + k], vm, k, -INFINITY));
+    }
+}
+
+// Largest value of the row: two independent accumulators, two new values per three-input
+// instruction.
+__device__ __forceinline__ float row_max(const uint32_t (&sv)[kKV]) {
+    float e0 = -INFINITY, e1 = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < kKV; k += 4) {
+        e0 = max3(e0, __uint_as_float(sv[k]), __uint_as_float(sv[k + 1]));
+        e1 = max3(e1, __uint_as_float(sv[k + 2]), __uint_as_float(sv[k + 3]));
+    }
+    return fmaxf(e0, e1);
+}
+
+// P = exp2(x + nm) of one row, packed to bf16 pairs and written over the first kKV/2 TMEM
+// columns of the row (32 S columns become 16 P columns, each chunk's P landing in columns
+// already read); returns the row sum of the fp32 values.  A -inf x gives 0.
+__device__ __forceinline__ float exp_row(const uint32_t (&sv)[kKV], uint32_t s_col, float nm) {
+    const uint64_t nm2 = f2_pack(nm, nm);
+    uint64_t l0 = f2_pack(0.f, 0.f), l1 = l0;
+#pragma unroll
+    for (int c = 0; c < kKV / 32; ++c) {
         uint32_t pk[16];
 #pragma unroll
-        for (int k = 0; k < 32; k += 4) {
-            float p0 = fast_exp2(fmaf(__uint_as_float(sv[c * 32 + k]), sce, nme));
-            float p1 = fast_exp2(fmaf(__uint_as_float(sv[c * 32 + k + 1]), sce, nme));
-            float p2 = fast_exp2(fmaf(__uint_as_float(sv[c * 32 + k + 2]), sce, nme));
-            float p3 = fast_exp2(fmaf(__uint_as_float(sv[c * 32 + k + 3]), sce, nme));
-            if (MASK) {
-                p0 = keep_or(__float_as_uint(p0), vm, k, 0.f);
-                p1 = keep_or(__float_as_uint(p1), vm, k + 1, 0.f);
-                p2 = keep_or(__float_as_uint(p2), vm, k + 2, 0.f);
-                p3 = keep_or(__float_as_uint(p3), vm, k + 3, 0.f);
-            }
-            l0 += p0;
-            l1 += p1;
-            l2 += p2;
-            l3 += p3;
-            pk[k / 2] = pack_bf16x2(p0, p1);
-            pk[k / 2 + 1] = pack_bf16x2(p2, p3);
+        for (int k = 0; k < 32; k += 2) {
+            float a, b;
+            f2_unpack(f2_add(f2_pack(__uint_as_float(sv[c * 32 + k]), __uint_as_float(sv[c * 32 + k + 1])), nm2), a, b);
+            a = fast_exp2(a);
+            b = fast_exp2(b);
+            const uint64_t p2 = f2_pack(a, b);
+            if ((k / 2) & 1)
+                l1 = f2_add(l1, p2);
+            else
+                l0 = f2_add(l0, p2);
+            pk[k / 2] = pack_bf16x2(a, b);
         }
         tmem_st16(s_col + c * 16, pk);
     }
-    return (l0 + l1) + (l2 + l3);
+    float a0, b0, a1, b1;
+    f2_unpack(l0, a0, b0);
+    f2_unpack(l1, a1, b1);
+    return (a0 + b0) + (a1 + b1);
 }
 
 struct PrefillParams {
@@ -203,6 +210,7 @@ struct Layout {
     static constexpr int BYTES = MISC_OFF + 16 + 4 * kUnitRing;
     static constexpr int ALLOC = BYTES + 1024;               // room to align the base to 1024
 };
+static_assert(Layout<128>::ALLOC <= 227 * 1024, "shared memory per CTA");
 
 struct TileInfo {
     bool valid;          // false: the pair's B slot is empty
@@ -442,7 +450,9 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
+    // (broadcast from lane 0: a shuffled value is known to be the same in every lane, which
+    // lets the compiler keep what is derived from it, like the MMA operands, warp-uniform)
+    const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
 
     // Work units: every plan entry for every head group.  In the shared-prefix mode the
     // work is small (a few groups' prefixes) and latency-bound, so each pair entry is
@@ -480,21 +490,15 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
         // key tile ahead so that no copy waits on a block-table lookup.
         uint32_t fill = 0;
         int qloads[2] = {0, 0};
-        int last_fill[kStages];
-        for (int s = 0; s < kStages; ++s) last_fill[s] = -1;
         const int piece = min(p.block_size, kKV);
+        // The block id of piece `lane` of key tile j, or kNoPiece for lanes past the tile's
+        // pieces.  The load is only issued here; its value is range-checked where it is
+        // used (load_kv, one key tile later), so the warp does not stall on it.
+        constexpr int kNoPiece = INT_MIN;
         auto load_pieces = [&](const int32_t* bt, int kbeg, int lk, int j) {
             const int key0 = j * kKV;
             const int npieces = (min(kKV, lk - key0) + piece - 1) / piece;
-            int blk = -1;
-            if (lane < npieces) {
-                blk = __ldg(bt + ((kbeg + key0 + lane * piece) >> p.block_shift));
-                if (blk < 0 || blk >= p.num_blocks) {
-                    flag_error(p.err, NVPA_FLAG_BAD_BLOCK_ID);
-                    blk = -1;
-                }
-            }
-            return blk;
+            return lane < npieces ? __ldg(bt + ((kbeg + key0 + lane * piece) >> p.block_shift)) : kNoPiece;
         };
         bool ok = true;
         for (int n = 0; ok; ++n) {
@@ -566,12 +570,15 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                 ++qloads[x];
                 return true;
             };
-            // K (kv = 0) or V tile j, whose block pieces lane c holds in blk_lane
+            // K (kv = 0) or V tile j, whose block pieces lane c holds in blk_lane; a block id out
+            // of range is flagged (once, with the K tile) and its piece is not loaded
             auto load_kv = [&](int kv, int j, int blk_lane) -> bool {
                 const int slot = fill % kStages;
                 if (!mbar_wait(bars + L::B_KVEMPTY + slot, ((fill / kStages) & 1) ^ 1, abort_flag, p.err))
                     return false;
-                const uint32_t valid_mask = __ballot_sync(0xffffffffu, blk_lane >= 0);
+                const bool in_range = blk_lane >= 0 && blk_lane < p.num_blocks;
+                if (kv == 0 && blk_lane != kNoPiece && !in_range) flag_error(p.err, NVPA_FLAG_BAD_BLOCK_ID);
+                const uint32_t valid_mask = __ballot_sync(0xffffffffu, in_range);
                 const uint32_t bytes = (uint32_t)__popc(valid_mask) * (uint32_t)(piece * 128 * L::REGIONS);
                 uint8_t* dst = smem + L::STAGE_OFF + slot * L::TILE_BYTES;
                 const CUtensorMap* map = kv ? &v_map : &k_map;
@@ -587,7 +594,6 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                                         r * 64, ta.hk, z);
                     }
                 }
-                last_fill[slot] = (int)fill;
                 ++fill;
                 return true;
             };
@@ -597,7 +603,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             if (ok && nkv > 0) ok = load_kv(0, 0, cur_blk);
             if (ok) ok = load_q(1);
             for (int j = 0; j < nkv && ok; ++j) {
-                const int nxt_blk = j + 1 < nkv ? load_pieces(bt, ta.kbeg, ta.lk, j + 1) : -1;
+                const int nxt_blk = j + 1 < nkv ? load_pieces(bt, ta.kbeg, ta.lk, j + 1) : kNoPiece;
                 if (j > 0) ok = load_kv(0, j, cur_blk);
                 if (ok) ok = load_kv(1, j, cur_blk);
                 cur_blk = nxt_blk;
@@ -605,10 +611,11 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
         }
         // let every copy this warp started land before the CTA can exit
         if (lane == 0) {
-            for (int s = 0; s < kStages; ++s) {
-                if (last_fill[s] < 0) continue;
+            for (uint32_t s = 0; s < (uint32_t)kStages; ++s) {
+                if (fill <= s) continue;
+                const uint32_t last = fill - 1 - (fill - 1 - s) % kStages;   // last fill of slot s
                 const uint64_t t0 = global_ns();
-                while (!mbar_try_wait(bars + L::B_KVFULL + s, (last_fill[s] / kStages) & 1) &&
+                while (!mbar_try_wait(bars + L::B_KVFULL + s, (last / kStages) & 1) &&
                        global_ns() - t0 < 100000000ull) {
                 }
             }
@@ -632,38 +639,45 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
         uint32_t puse[2] = {0, 0};             // P_j waits per tile
         int units[2] = {0, 0};                 // units in which the tile had work
         bool ok = true;
+        // Operand descriptors: one low half per buffer (Q tiles and ring stage 0, K-major for
+        // S, MN-major for V), offsets added per MMA; every operand of the MMA instructions
+        // is derived from warp-uniform values only, so issuing one costs a few instructions.
+        constexpr uint32_t DESC_HI = sdesc_sw128_hi(1024);
+        constexpr uint32_t TILE16 = L::TILE_BYTES >> 4, REGION16 = L::REGION_BYTES >> 4;
+        const uint32_t q_lo = sdesc_sw128_lo(sbase + L::Q_OFF, 16);
+        const uint32_t k_lo = sdesc_sw128_lo(sbase + L::STAGE_OFF, 16);
+        const uint32_t v_lo = sdesc_sw128_lo(sbase + L::STAGE_OFF, L::REGION_BYTES);
         auto issue_qk = [&](int x, int kslot) {
-            const uint32_t q_addr = sbase + L::Q_OFF + x * L::TILE_BYTES;
-            const uint32_t k_addr = sbase + L::STAGE_OFF + kslot * L::TILE_BYTES;
+            const uint32_t a = q_lo + (uint32_t)x * TILE16, b = k_lo + (uint32_t)kslot * TILE16;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-                const int r = kk / 4, off = (kk % 4) * 32;
-                const uint64_t adesc = sdesc_sw128(q_addr + r * L::REGION_BYTES + off, 16, 1024);
-                const uint64_t bdesc = sdesc_sw128(k_addr + r * L::REGION_BYTES + off, 16, 1024);
-                umma_ss(tmem + x * 256, adesc, bdesc, IDESC_QK, kk > 0 ? 1u : 0u);
+                const uint32_t o = (kk / 4) * REGION16 + (kk % 4) * 2;   // 64-column region, 32 bytes of K
+                umma_ss(tmem + x * 256, sdesc_join(a + o, DESC_HI), sdesc_join(b + o, DESC_HI), IDESC_QK,
+                        kk > 0 ? 1u : 0u);
             }
             umma_commit(bars + L::B_SFULL + x);
         };
         auto issue_pv = [&](int x, int vslot, bool accumulate) {
-            const uint32_t v_addr = sbase + L::STAGE_OFF + vslot * L::TILE_BYTES;
+            const uint32_t b = v_lo + (uint32_t)vslot * TILE16;
 #pragma unroll
-            for (int kk = 0; kk < kKV / 16; ++kk) {
-                const uint64_t bdesc = sdesc_sw128(v_addr + kk * 16 * 128, L::REGION_BYTES, 1024);
-                umma_ts(tmem + x * 256 + kKV, tmem + x * 256 + kk * 8, bdesc, IDESC_PV,
+            for (int kk = 0; kk < kKV / 16; ++kk)   // 16 keys = 16 rows of 128 bytes per MMA
+                umma_ts(tmem + x * 256 + kKV, tmem + x * 256 + kk * 8, sdesc_join(b + kk * 128, DESC_HI), IDESC_PV,
                         (accumulate || kk > 0) ? 1u : 0u);
-            }
             umma_commit(bars + L::B_ODONE + x);
         };
         for (int n = 0; ok; ++n) {
-            const int idx = claim(n);
+            const int idx = __shfl_sync(0xffffffffu, claim(n), 0);
             if (idx < 0) break;
             int4 e;
             int hg;
             unit_of(idx, e, hg);
             const TileInfo ta = tile_info<PREFIX>(p, e, hg, false);
             const TileInfo tb = tile_info<PREFIX>(p, e, hg, true);
-            const int nk[2] = {ta.nkv, tb.nkv};
-            const bool val[2] = {ta.valid, tb.valid};
+            // the ring positions follow from these counts: broadcast them (see tmem above)
+            const int nk[2] = {__shfl_sync(0xffffffffu, ta.nkv, 0), __shfl_sync(0xffffffffu, tb.nkv, 0)};
+            const bool val[2] = {__shfl_sync(0xffffffffu, (int)ta.valid, 0) != 0,
+                                 __shfl_sync(0xffffffffu, (int)tb.valid, 0) != 0};
+            const int lk = __shfl_sync(0xffffffffu, ta.lk, 0);
             const int nkv = max(nk[0], nk[1]);
             // S of key tile 0: tile A as soon as Q_A and K_0 are in, then tile B
             if (nkv > 0 && !mbar_wait(bars + L::B_KVFULL + fbase % kStages, (fbase / kStages) & 1, abort_flag, p.err))
@@ -691,7 +705,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                     ok = false;
                     break;
                 }
-                const int valid = min(kKV, ta.lk - j * kKV);
+                const int valid = min(kKV, lk - j * kKV);
                 if (valid < kKV) {
                     // zero the V rows past the sequence (stale cache rows, or never loaded)
                     uint8_t* vt = smem + L::STAGE_OFF + vslot * L::TILE_BYTES;
@@ -716,23 +730,28 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                         ok = false;
                         break;
                     }
-                    if (j + 1 < nk[x] && !k_next) {
-                        if (!mbar_wait(bars + L::B_KVFULL + kslot, (fk / kStages) & 1, abort_flag, p.err)) {
-                            ok = false;
-                            break;
-                        }
-                        k_next = true;
-                    }
                     tc_fence_after();
+                    // P V first: it does not need K_{j+1}, which may still be in flight
                     if (lane == 0) {
                         issue_pv(x, vslot, j > 0);
                         if (j == nk[x] - 1) umma_commit(bars + L::B_OFINAL + x);
-                        if (j + 1 < nk[x]) {
+                    }
+                    __syncwarp();
+                    if (j + 1 < nk[x]) {
+                        if (!k_next) {
+                            if (!mbar_wait(bars + L::B_KVFULL + kslot, (fk / kStages) & 1, abort_flag, p.err)) {
+                                ok = false;
+                                break;
+                            }
+                            k_next = true;
+                            tc_fence_after();
+                        }
+                        if (lane == 0) {
                             issue_qk(x, kslot);
                             if (j + 2 == nk[x]) umma_commit(bars + L::B_QEMPTY + x);
                         }
+                        __syncwarp();
                     }
-                    __syncwarp();
                 }
                 if (!ok) break;
                 if (lane == 0) {
@@ -802,17 +821,11 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                 for (int c = 0; c < kKV / 32; ++c)
                     tmem_ld32(s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
                 tmem_wait_ld();
-                // pass 1: the row's largest visible scaled score: the max of the raw scores
-                // for a positive scale, the min for a negative one.  The softmax is bound by
-                // the ALU pipe (min/max, selects, packing), so tiles that need no mask take a
-                // loop of three-input max/min and nothing else.
-                const float sc = p.scale_log2;
-                float ext;
-                if (open)
-                    ext = sc >= 0.f ? row_extreme<true, false>(sv, key0, lim) : row_extreme<false, false>(sv, key0, lim);
-                else
-                    ext = sc >= 0.f ? row_extreme<true, true>(sv, key0, lim) : row_extreme<false, true>(sv, key0, lim);
-                const float mt = fabsf(ext) == INFINITY ? -INFINITY : ext * sc;
+                // scaled scores, keys the row does not see at -inf (diagonal tiles only),
+                // then the row's largest value
+                scale_row(sv, p.scale_log2);
+                if (!open) mask_row(sv, key0, lim);
+                const float mt = row_max(sv);
                 const bool over = mt > m + kRescaleSlack;
                 const bool rescale = __any_sync(0xffffffffu, over);
                 float alpha = 1.f;
@@ -822,13 +835,9 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                     l *= alpha;
                     m = m_new;
                 }
-                // pass 2: P_j = exp2(s * scale - m) as bf16 pairs over the first kKV/2 columns
-                // of S_j.  A row with no visible key yet (m = -inf) gets exp2(-inf) = 0
-                // through its operands, not through a select per element.
-                const bool live = m > -INFINITY;
-                const float sce = live ? sc : 0.f, nme = live ? -m : -INFINITY;
-                l += open ? exp_row<false>(sv, s_col, sce, nme, key0, lim)
-                          : exp_row<true>(sv, s_col, sce, nme, key0, lim);
+                // P_j = exp2(x - m) as bf16 pairs over the first kKV/2 columns of S_j.  A row
+                // with no visible key yet (m = -inf) gets exp2(-inf) = 0 through its offset.
+                l += exp_row(sv, s_col, m > -INFINITY ? -m : -INFINITY);
                 if (rescale && j > 0) {
                     // O holds P_0..P_{j-1} V (all complete once S_j is): rescale it before
                     // P_j is released to the MMA

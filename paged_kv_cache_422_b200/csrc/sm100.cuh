@@ -180,13 +180,33 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand: start address,
 // leading- and stride-dimension byte offsets (16-byte units), sm_100 descriptor version 1,
 // layout type SWIZZLE_128B.  Swizzle atoms must be 1024-byte aligned.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+__host__ __device__ constexpr uint64_t sdesc_sw128(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
     return (uint64_t)((smem_addr >> 4) & 0x3FFFu)
          | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16)
          | ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32)
          | (1ull << 46)
          | (2ull << 61);
 }
+
+// The same descriptor as two 32-bit halves: the low half holds the start address and the
+// leading-dimension offset, the high half everything else.  Adding (byte offset >> 4) to
+// the low half moves the start address (16-byte aligned offsets, addresses below 256 KB,
+// so nothing carries out of the 14-bit address field); an MMA loop can then keep one low
+// half per buffer and add compile-time offsets.
+__host__ __device__ constexpr uint32_t sdesc_sw128_lo(uint32_t smem_addr, uint32_t lbo_bytes) {
+    return ((smem_addr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ constexpr uint32_t sdesc_sw128_hi(uint32_t sbo_bytes) {
+    return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+}
+__host__ __device__ constexpr uint64_t sdesc_join(uint32_t lo, uint32_t hi) {
+    return ((uint64_t)hi << 32) | lo;
+}
+static_assert(sdesc_join(sdesc_sw128_lo(0x2c400u, 16u), sdesc_sw128_hi(1024u)) == sdesc_sw128(0x2c400u, 16u, 1024u),
+              "descriptor halves");
+static_assert(sdesc_join(sdesc_sw128_lo(0x8000u, 16384u) + 0x80u, sdesc_sw128_hi(1024u)) ==
+                  sdesc_sw128(0x8800u, 16384u, 1024u),
+              "descriptor offset");
 
 // D[tmem] (+)= A[smem] * B[smem]
 __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
