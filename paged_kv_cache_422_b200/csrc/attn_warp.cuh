@@ -45,11 +45,6 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
 // A packed bf16 pair (low half = element 2j, high half = element 2j+1) widened exactly.
 __device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
     return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));

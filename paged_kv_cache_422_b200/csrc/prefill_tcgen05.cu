@@ -18,7 +18,7 @@
 // each tile is fetched once for 256 query rows, and the two tiles' MMAs and softmaxes
 // interleave: while one tile's softmax runs, the tensor core computes the other tile's
 // P V and its next S.  One CTA per SM (persistent; CTA c takes units c, c + grid, ...);
-// the plan kernel lists the pairs, heaviest sequences first.  Warp roles:
+// the plan kernel lists the pairs, most key tiles first.  Warp roles:
 //   warp 0      TMA producer: Q_A, K_0, Q_B, V_0, then K_j and V_j tiles into a 5-stage
 //               ring (one 3-D tensor-map box per cache block piece; a 128-key tile spans
 //               128 / block_size blocks when the block size is below 128).  Q_B's buffer
@@ -84,6 +84,12 @@ __device__ __forceinline__ uint32_t visible_mask(int n) {
 __device__ __forceinline__ float keep_or(uint32_t bits, uint32_t vm, int k, float fill) {
     const uint32_t keep = (uint32_t)((int32_t)(vm << (31 - k)) >> 31);
     return __uint_as_float((bits & keep) | (__float_as_uint(fill) & ~keep));
+}
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
 }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
@@ -206,11 +212,22 @@ struct Layout {
     static constexpr int B_OFINAL = B_ODONE + 2, B_OFREE = B_OFINAL + 2, B_DRAIN = B_OFREE + 2;
     static constexpr int B_UFULL = B_DRAIN + 1, B_UEMPTY = B_UFULL + kUnitRing;
     static constexpr int NBARS = B_UEMPTY + kUnitRing;
-    static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;     // tmem base, abort flag, unit ring
-    static constexpr int BYTES = MISC_OFF + 16 + 4 * kUnitRing;
+    static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;     // tmem base, abort flag
+    static constexpr int RING_OFF = (MISC_OFF + 16 + 15) / 16 * 16;   // unit descriptions
+    static constexpr int BYTES = RING_OFF + 32 * kUnitRing;
     static constexpr int ALLOC = BYTES + 1024;               // room to align the base to 1024
 };
 static_assert(Layout<128>::ALLOC <= 227 * 1024, "shared memory per CTA");
+
+// A work unit as the producer hands it to the MMA and softmax warps (32 bytes in shared
+// memory): its plan entry, head group and the lengths of its sequence (or prefix group),
+// so that no consumer reads global memory at a unit boundary.  e.x < 0 ends the loop.
+struct UnitDesc {
+    int4 e;              // plan entry: sequence (group), query tile A, tile B or -1, key partition
+    int hg;              // head group
+    int q0, lq, lk;      // first query row, query rows, keys (prefix mode: prefix length)
+};
+static_assert(sizeof(UnitDesc) == 32, "unit description size");
 
 struct TileInfo {
     bool valid;          // false: the pair's B slot is empty
@@ -226,30 +243,28 @@ __device__ __forceinline__ int tile_nkv(int causal, int lq, int lk, int tok0, in
     return causal ? min(ktiles, (lk - lq + tok0 + ntok - 1) / kKV + 1) : ktiles;
 }
 
-// Tile A (second = false) or B of plan entry e for head group hg.
+// Tile A (second = false) or B of unit u.
 template <bool PREFIX>
-__device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, int4 e, int hg, bool second) {
+__device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, const UnitDesc& u, bool second) {
     TileInfo t;
-    const int qt = second ? e.z : e.y;
+    const int qt = second ? u.e.z : u.e.y;
     t.valid = qt >= 0;
-    t.seq = e.x;
+    t.seq = u.e.x;
     t.qt = max(qt, 0);
-    t.head0 = hg * p.pack;
+    t.head0 = u.hg * p.pack;
     t.hk = t.head0 / p.group;
+    t.q0 = u.q0;
+    t.lq = u.lq;
     if constexpr (PREFIX) {
         // group e.x: its members are the queries, keys [kbeg, kbeg + lk) of its shared
         // prefix the keys (no mask)
-        t.chunk = e.w;
+        t.chunk = u.e.w;
         t.kbeg = t.chunk * p.pchunk;
-        t.q0 = __ldg(p.group_start + t.seq);
-        t.lq = __ldg(p.group_start + t.seq + 1) - t.q0;
-        t.lk = min(p.pchunk, __ldg(p.group_len + t.seq) - t.kbeg);
+        t.lk = min(p.pchunk, u.lk - t.kbeg);
     } else {
         t.chunk = 0;
         t.kbeg = 0;
-        t.q0 = __ldg(p.cu_q + t.seq);
-        t.lq = __ldg(p.cu_q + t.seq + 1) - t.q0;
-        t.lk = __ldg(p.cu_k + t.seq + 1) - __ldg(p.cu_k + t.seq);
+        t.lk = u.lk;
     }
     t.tok0 = t.qt * p.tq;
     t.ntok = min(p.tq, t.lq - t.tok0);
@@ -257,33 +272,52 @@ __device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, int4 e, in
     return t;
 }
 
-// ------------------------------------------------------------------------------------
-// plan: list the query-tile pairs, the sequences with the most key tiles first
-// ------------------------------------------------------------------------------------
-constexpr int kPlanMaxRanked = 2048;   // batches up to this size are ordered by sequence
-
-// Entries are grouped by sequence, sequences with the most work (key tiles visited over
-// all their query tiles) first and, inside a sequence, the pairs with the most key tiles
-// first.  CTAs that run at the same time then mostly read the same sequences' keys and
-// values, which L2 serves after the first fetch, and the longest work starts first.  A
-// sequence with cnt query tiles gives the pairs (2w, 2w+1) counted from its first tile,
-// last pair first; for odd cnt the last tile stands alone.  Counting from the first tile
-// aligns a pair with the 128-key tiles when 2 * tokens per tile = 128 and the cached
-// prefix is a whole number of 128-key tiles (block sizes of 128 and 256): both tiles of
-// a pair then end in the same key tile and finish their key loops together.
-__device__ __forceinline__ void write_pairs(int4* tiles, int off, int seq, int cnt) {
-    const int npairs = (cnt + 1) / 2;
-    for (int u = 0; u < npairs; ++u) {
-        const int w = npairs - 1 - u;
-        tiles[off + u] = make_int4(seq, 2 * w, 2 * w + 1 < cnt ? 2 * w + 1 : -1, 0);
+// The lengths of the sequence (group) of plan entry e, from global memory.
+template <bool PREFIX>
+__device__ __forceinline__ UnitDesc describe_unit(const PrefillParams& p, int4 e, int hg) {
+    UnitDesc u;
+    u.e = e;
+    u.hg = hg;
+    if (e.x < 0) {
+        u.q0 = u.lq = u.lk = 0;
+    } else if constexpr (PREFIX) {
+        u.q0 = __ldg(p.group_start + e.x);
+        u.lq = __ldg(p.group_start + e.x + 1) - u.q0;
+        u.lk = __ldg(p.group_len + e.x);
+    } else {
+        u.q0 = __ldg(p.cu_q + e.x);
+        u.lq = __ldg(p.cu_q + e.x + 1) - u.q0;
+        u.lk = __ldg(p.cu_k + e.x + 1) - __ldg(p.cu_k + e.x);
     }
+    return u;
 }
 
+// ------------------------------------------------------------------------------------
+// plan: list the query-tile pairs, the ones with the most key tiles first
+// ------------------------------------------------------------------------------------
+constexpr int kPlanBuckets = 4096;   // key-tile counts sorted exactly; longer pairs share the top bucket
+
+// Key tiles visited by the pair (2w, 2w + 1) of a sequence with cnt query tiles (tile
+// 2w + 1, when it exists, ends later and visits at least as many).
+__device__ __forceinline__ int pair_nkv(const PrefillParams& p, int lq, int lk, int cnt, int w) {
+    const int qt = 2 * w + 1 < cnt ? 2 * w + 1 : 2 * w;
+    return tile_nkv(p.causal, lq, lk, qt * p.tq, min(p.tq, lq - qt * p.tq));
+}
+
+// Work units are pairs of query tiles (2w, 2w + 1) of one sequence, counted from its first
+// tile, so that both tiles of a pair end in the same 128-key tile when 2 * tokens per tile
+// = 128 and the cached prefix is a whole number of 128-key tiles (block sizes 128 and
+// 256): they then finish their key loops together; for an odd tile count the last tile
+// stands alone.  The list is sorted by key tiles, most first (a counting sort over the
+// pairs' key-tile counts), so that the units claimed last are the shortest and the CTAs
+// finish close together.  The order inside one count is whatever the atomics give: it
+// decides only which CTA runs a unit, never a result.
 __global__ void __launch_bounds__(1024) prefill_plan_kernel(const PrefillParams p, int4* tiles,
                                                             int32_t* ntiles) {
-    __shared__ int s_work[kPlanMaxRanked];
-    __shared__ int s_count[kPlanMaxRanked];
+    __shared__ int s_hist[kPlanBuckets];
     __shared__ int warp_tot[32];
+    // the attention grid may launch now: it sets up, then waits for this grid to complete
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const long long cap = (long long)p.max_blocks * p.block_size;
     auto seq_ok = [&](int i, int& lq, int& lk) {
@@ -294,100 +328,68 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const PrefillParams 
         return q0 >= 0 && lq >= 0 && lk >= lq && lq <= p.max_q && lk <= p.max_k && lk <= cap &&
                q1 <= p.total_q;
     };
-    const int nb = min(p.batch, kPlanMaxRanked);
-    // per sequence: pairs and work (nothing for a malformed sequence, which is flagged)
-    for (int i = tid; i < kPlanMaxRanked; i += blockDim.x) {
-        int lq = 0, lk = 0, cnt = 0, work = 0;
-        if (i < p.batch) {
-            if (seq_ok(i, lq, lk)) {
-                cnt = (lq + p.tq - 1) / p.tq;
-                for (int qt = 0; qt < cnt; ++qt)
-                    work += tile_nkv(p.causal, lq, lk, qt * p.tq, min(p.tq, lq - qt * p.tq));
-            } else {
-                flag_error(p.err, NVPA_FLAG_BAD_LENGTH);
-            }
+    auto bucket = [&](int nkv) { return min(nkv, kPlanBuckets - 1); };
+    for (int b = tid; b < kPlanBuckets; b += blockDim.x) s_hist[b] = 0;
+    __syncthreads();
+    // histogram of the pairs' key-tile counts (a malformed sequence gives none and is flagged)
+    for (int i = tid; i < p.batch; i += blockDim.x) {
+        int lq, lk;
+        if (!seq_ok(i, lq, lk)) {
+            flag_error(p.err, NVPA_FLAG_BAD_LENGTH);
+            continue;
         }
-        if (i < nb) {
-            s_work[i] = work;
-            s_count[i] = (cnt + 1) / 2;
-        }
+        const int cnt = (lq + p.tq - 1) / p.tq;
+        for (int w = 0; 2 * w < cnt; ++w) atomicAdd(&s_hist[bucket(pair_nkv(p, lq, lk, cnt, w))], 1);
     }
     __syncthreads();
-    // rank of each of the first nb sequences: heavier first, ties by index
-    int rank_of[kPlanMaxRanked / 1024];
-    for (int k = 0; k < kPlanMaxRanked / 1024; ++k) {
-        const int i = tid + k * 1024;
-        int rnk = 0;
-        if (i < nb) {
-            const int wi = s_work[i];
-            for (int jj = 0; jj < nb; ++jj) {
-                const int wj = s_work[jj];
-                rnk += (wj > wi || (wj == wi && jj < i)) ? 1 : 0;
-            }
-        }
-        rank_of[k] = rnk;
+    // first position of each count, counts in descending order: thread t takes buckets
+    // kPlanBuckets - 1 - 4t - k (k < 4); a block-wide exclusive scan of the thread sums
+    constexpr int kPer = kPlanBuckets / 1024;
+    int v[kPer];
+    int sum = 0;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        v[k] = s_hist[kPlanBuckets - 1 - (kPer * tid + k)];
+        sum += v[k];
     }
-    __syncthreads();
-    // reorder the pair counts by rank (reuse s_work as counts-in-rank-order)
-    for (int k = 0; k < kPlanMaxRanked / 1024; ++k) {
-        const int i = tid + k * 1024;
-        if (i < nb) s_work[rank_of[k]] = s_count[i];
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
     }
+    if (lane == 31) warp_tot[wid] = incl;
     __syncthreads();
-    // exclusive prefix over ranks (two 1024-element passes)
-    int carry = 0;
-    for (int k = 0; k < kPlanMaxRanked / 1024; ++k) {
-        const int r = tid + k * 1024;
-        int v = r < nb ? s_work[r] : 0;
-        int incl = v;
+    if (wid == 0) {
+        int w = warp_tot[lane];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += n;
+            const int n = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += n;
         }
-        if (lane == 31) warp_tot[wid] = incl;
-        __syncthreads();
-        if (wid == 0) {
-            int w = warp_tot[lane];
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int n = __shfl_up_sync(0xffffffffu, w, o);
-                if (lane >= o) w += n;
-            }
-            warp_tot[lane] = w;
-        }
-        __syncthreads();
-        const int excl = carry + incl - v + (wid ? warp_tot[wid - 1] : 0);
-        const int block_total = warp_tot[31];
-        __syncthreads();
-        if (r < nb) s_count[r] = excl;   // s_count now: offset of rank r
-        carry += block_total;
+        warp_tot[lane] = w;
     }
     __syncthreads();
-    int written = carry;
-    for (int k = 0; k < kPlanMaxRanked / 1024; ++k) {
-        const int i = tid + k * 1024;
-        if (i >= nb) continue;
+    int run = incl - sum + (wid ? warp_tot[wid - 1] : 0);
+    const int total = warp_tot[31];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        s_hist[kPlanBuckets - 1 - (kPer * tid + k)] = run;
+        run += v[k];
+    }
+    __syncthreads();
+    // place each pair at the next free position of its count
+    for (int i = tid; i < p.batch; i += blockDim.x) {
         int lq, lk;
         if (!seq_ok(i, lq, lk)) continue;
-        write_pairs(tiles, s_count[rank_of[k]], i, (lq + p.tq - 1) / p.tq);
-    }
-    // sequences beyond the ranked ones (very large batches) follow in index order
-    if (p.batch > nb) {
-        __shared__ int extra_base;
-        if (tid == 0) extra_base = written;
-        __syncthreads();
-        for (int i = nb + tid; i < p.batch; i += blockDim.x) {
-            int lq, lk;
-            if (!seq_ok(i, lq, lk)) continue;
-            const int cnt = (lq + p.tq - 1) / p.tq;
-            write_pairs(tiles, atomicAdd(&extra_base, (cnt + 1) / 2), i, cnt);
+        const int cnt = (lq + p.tq - 1) / p.tq;
+        for (int w = 0; 2 * w < cnt; ++w) {
+            const int pos = atomicAdd(&s_hist[bucket(pair_nkv(p, lq, lk, cnt, w))], 1);
+            tiles[pos] = make_int4(i, 2 * w, 2 * w + 1 < cnt ? 2 * w + 1 : -1, 0);
         }
-        __syncthreads();
-        if (tid == 0) written = extra_base;
     }
     if (tid == 0) {
-        *ntiles = written;
+        *ntiles = total;
         ntiles[1] = 0;   // the attention kernel's unit counter
     }
 }
@@ -408,14 +410,12 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
-    volatile int* unit_ring = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 16);
+    UnitDesc* unit_ring = reinterpret_cast<UnitDesc*>(smem + L::RING_OFF);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if constexpr (PREFIX) {
-        // shared-prefix mode follows the decode plan: let the worker's CTAs launch as this
-        // grid's CTAs finish, and wait for the plan's tables
+        // shared-prefix mode: let the decode worker's CTAs launch as this grid's CTAs finish
         asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-        asm volatile("griddepcontrol.wait;" ::: "memory");
     }
 
     if (threadIdx.x == 0) {
@@ -453,6 +453,9 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
     // (broadcast from lane 0: a shuffled value is known to be the same in every lane, which
     // lets the compiler keep what is derived from it, like the MMA operands, warp-uniform)
     const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
+    // This grid is launched as a programmatic dependent of its plan kernel: the setup above
+    // overlaps the plan, and nothing the plan writes is read before this wait.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // Work units: every plan entry for every head group.  In the shared-prefix mode the
     // work is small (a few groups' prefixes) and latency-bound, so each pair entry is
@@ -468,16 +471,22 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
         }
     };
     // Units are claimed dynamically (longest first, as the plan orders them): the producer
-    // claims the next one with an atomic and hands its index to the MMA and softmax warps
-    // through a small ring in shared memory; -1 ends the loop.  claim(n) returns the n-th
-    // unit of this CTA, -1 at the end, -2 if a wait timed out.
-    auto claim = [&](int n) -> int {
+    // claims them with an atomic, one unit ahead of the one it loads, and hands each one's
+    // description to the MMA and softmax warps through a small ring in shared memory.
+    // claim(n) returns the n-th unit of this CTA; e.x is -1 at the end, -2 if a wait timed
+    // out.
+    auto claim = [&](int n) -> UnitDesc {
         const int slot = n % kUnitRing;
-        if (!mbar_wait(bars + L::B_UFULL + slot, (n / kUnitRing) & 1, abort_flag, p.err)) return -2;
-        const int idx = unit_ring[slot];
+        UnitDesc u;
+        if (!mbar_wait(bars + L::B_UFULL + slot, (n / kUnitRing) & 1, abort_flag, p.err)) {
+            u.e = make_int4(-2, -1, -1, 0);
+            u.hg = u.q0 = u.lq = u.lk = 0;
+            return u;
+        }
+        u = unit_ring[slot];
         __syncwarp();
         if (lane == 0) mbar_arrive(bars + L::B_UEMPTY + slot);
-        return idx;
+        return u;
     };
 
     if (warp < 4) {
@@ -500,28 +509,49 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             const int npieces = (min(kKV, lk - key0) + piece - 1) / piece;
             return lane < npieces ? __ldg(bt + ((kbeg + key0 + lane * piece) >> p.block_shift)) : kNoPiece;
         };
+        // Claims run one unit ahead: the index and description of unit n + 1 are fetched
+        // while unit n's copies are issued, so that the next unit's first copies do not
+        // wait for an atomic and two dependent global loads.
+        auto claim_next = [&]() -> int { return lane == 0 ? atomicAdd(p.unit_counter, 1) : 0; };
+        auto resolve = [&](int pending) -> int {
+            const int i = __shfl_sync(0xffffffffu, pending, 0);
+            return i < total ? i : -1;
+        };
+        auto entry = [&](int idx, int4& e, int& hg) {
+            e = make_int4(-1, -1, -1, 0);
+            hg = 0;
+            if (idx >= 0) unit_of(idx, e, hg);
+        };
+        UnitDesc cur;
+        {
+            int4 e;
+            int hg;
+            entry(resolve(claim_next()), e, hg);
+            cur = describe_unit<PREFIX>(p, e, hg);
+        }
+        int pending = claim_next();
         bool ok = true;
         for (int n = 0; ok; ++n) {
             const int slot = n % kUnitRing;
             if (!mbar_wait(bars + L::B_UEMPTY + slot, ((n / kUnitRing) & 1) ^ 1, abort_flag, p.err)) break;
-            int idx = 0;
             if (lane == 0) {
-                idx = atomicAdd(p.unit_counter, 1);
-                if (idx >= total) idx = -1;
-                unit_ring[slot] = idx;
+                unit_ring[slot] = cur;
                 mbar_arrive(bars + L::B_UFULL + slot);
             }
-            idx = __shfl_sync(0xffffffffu, idx, 0);
-            if (idx < 0) break;
-            int4 e;
-            int hg;
-            unit_of(idx, e, hg);
-            const TileInfo ta = tile_info<PREFIX>(p, e, hg, false);
-            const TileInfo tb = tile_info<PREFIX>(p, e, hg, true);
+            if (cur.e.x < 0) break;
+            // the next unit: its index now, its plan entry in flight, and the claim after it
+            const int nidx = resolve(pending);
+            int4 ne;
+            int nhg;
+            entry(nidx, ne, nhg);
+            pending = nidx >= 0 ? claim_next() : total;
+            const TileInfo ta = tile_info<PREFIX>(p, cur, false);
+            const TileInfo tb = tile_info<PREFIX>(p, cur, true);
             const int nkv = max(ta.nkv, tb.nkv);
             const int bt_seq = PREFIX ? __ldg(p.members + ta.q0) : ta.seq;   // a member's table
             const int32_t* bt = p.block_tables + (size_t)bt_seq * p.max_blocks;
             int cur_blk = load_pieces(bt, ta.kbeg, ta.lk, 0);
+            int nxt_blk = nkv > 1 ? load_pieces(bt, ta.kbeg, ta.lk, 1) : kNoPiece;
             // Q tile x of this unit (its buffer frees after the last S of the previous unit's
             // tile x)
             auto load_q = [&](int x) -> bool {
@@ -597,17 +627,22 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                 ++fill;
                 return true;
             };
-            // Q_A, K_0, Q_B, V_0, then K_j, V_j: tile B's Q buffer frees last (B has the most
-            // key tiles), so K_0 and tile A's first S do not wait for it
-            ok = load_q(0);
-            if (ok && nkv > 0) ok = load_kv(0, 0, cur_blk);
+            // K_0 first (its ring slot frees early), then Q_A (its buffer frees when the
+            // previous unit's last S of tile A completes), V_0 and Q_B (frees last: tile B has
+            // the most key tiles), then K_j, V_j
+            if (nkv > 0) ok = load_kv(0, 0, cur_blk);
+            if (ok) ok = load_q(0);
+            if (ok && nkv > 0) ok = load_kv(1, 0, cur_blk);
             if (ok) ok = load_q(1);
-            for (int j = 0; j < nkv && ok; ++j) {
-                const int nxt_blk = j + 1 < nkv ? load_pieces(bt, ta.kbeg, ta.lk, j + 1) : kNoPiece;
-                if (j > 0) ok = load_kv(0, j, cur_blk);
-                if (ok) ok = load_kv(1, j, cur_blk);
+            // the lengths of the next unit's sequence: these loads overlap this unit's waits
+            const UnitDesc nxt = describe_unit<PREFIX>(p, ne, nhg);
+            for (int j = 1; j < nkv && ok; ++j) {
                 cur_blk = nxt_blk;
+                nxt_blk = j + 1 < nkv ? load_pieces(bt, ta.kbeg, ta.lk, j + 1) : kNoPiece;
+                ok = load_kv(0, j, cur_blk);
+                if (ok) ok = load_kv(1, j, cur_blk);
             }
+            cur = nxt;
         }
         // let every copy this warp started land before the CTA can exit
         if (lane == 0) {
@@ -666,13 +701,10 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             umma_commit(bars + L::B_ODONE + x);
         };
         for (int n = 0; ok; ++n) {
-            const int idx = __shfl_sync(0xffffffffu, claim(n), 0);
-            if (idx < 0) break;
-            int4 e;
-            int hg;
-            unit_of(idx, e, hg);
-            const TileInfo ta = tile_info<PREFIX>(p, e, hg, false);
-            const TileInfo tb = tile_info<PREFIX>(p, e, hg, true);
+            const UnitDesc u = claim(n);
+            if (__shfl_sync(0xffffffffu, u.e.x, 0) < 0) break;
+            const TileInfo ta = tile_info<PREFIX>(p, u, false);
+            const TileInfo tb = tile_info<PREFIX>(p, u, true);
             // the ring positions follow from these counts: broadcast them (see tmem above)
             const int nk[2] = {__shfl_sync(0xffffffffu, ta.nkv, 0), __shfl_sync(0xffffffffu, tb.nkv, 0)};
             const bool val[2] = {__shfl_sync(0xffffffffu, (int)ta.valid, 0) != 0,
@@ -794,12 +826,9 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
         int tcount = 0;
         uint32_t pv_before = 0;                       // PVs issued for this tile slot before
         for (int n = 0;; ++n) {
-            const int idx = claim(n);
-            if (idx < 0) break;
-            int4 e;
-            int hg;
-            unit_of(idx, e, hg);
-            const TileInfo t = tile_info<PREFIX>(p, e, hg, x == 1);
+            const UnitDesc u = claim(n);
+            if (u.e.x < 0) break;
+            const TileInfo t = tile_info<PREFIX>(p, u, x == 1);
             if (t.nkv == 0) continue;
             const int pos = t.lk - t.lq + t.tok0 + rtok;           // absolute position of this row
             const int lim = (!PREFIX && p.causal) ? min(t.lk, pos + 1) : t.lk;  // keys 0 .. lim-1 visible
@@ -1096,8 +1125,8 @@ nvpa_status_t run_varlen_prefill_tcgen05(const PrefillCall& c, void* workspace, 
     // one pair per query tile at most, plus one per sequence for a ragged last tile
     const long long max_units = ((long long)c.batch + (c.total_q + p.tq - 1) / p.tq) * p.hgroups;
     const int grid = (int)std::max(1LL, std::min<long long>((long long)device_sm_count(), max_units));
-    e = c.head_dim == 128 ? launch_prefill<128, false>(qm, km, vm, p, grid, stream)
-                          : launch_prefill<64, false>(qm, km, vm, p, grid, stream);
+    e = c.head_dim == 128 ? launch_prefill<128, false>(qm, km, vm, p, grid, stream, true)
+                          : launch_prefill<64, false>(qm, km, vm, p, grid, stream, true);
     if (e != cudaSuccess) return cuda_failure(e, "prefill tcgen05 launch");
     count_launches(1);
     return NVPA_OK;
