@@ -280,6 +280,31 @@ def cpu_baseline(step, budget_s: float = 12.0) -> dict:
                        f"{tot_t:.1f} s; seq-steps/s {n / tot_t:.3f}")
 
 
+def prefill_cpu_baseline(step, budget_s: float = 10.0) -> dict:
+    """The oracle's varlen prefill on as many whole sequences (in a fixed shuffled order) as
+    fit in about budget_s seconds; TFLOP/s counts the sample's algorithmic causal FLOPs."""
+    import oracle
+    kc, vc = step.k_pool.copy(), step.v_pool.copy()
+    oracle.store_kvcache(kc, vc, step.k_new, step.v_new, step.slot_mapping)
+    d, hq = step.head_dim, step.num_q_heads
+    order = np.random.default_rng(0).permutation(step.batch)
+    tot_t, tot_f, n = 0.0, 0, 0
+    while n < step.batch and tot_t < budget_s:
+        i = int(order[n])
+        q0, q1 = int(step.cu_seqlens_q[i]), int(step.cu_seqlens_q[i + 1])
+        lq, lk = q1 - q0, int(step.cu_seqlens_k[i + 1] - step.cu_seqlens_k[i])
+        t0 = time.perf_counter()
+        oracle.varlen_prefill_attention(step.q[q0:q1], kc, vc, step.block_tables[i:i + 1],
+                                        np.array([0, lq], np.int32), np.array([0, lk], np.int32),
+                                        step.scale)
+        tot_t += time.perf_counter() - t0
+        tot_f += 4 * d * hq * (lq * (lk - lq) + lq * (lq + 1) // 2)
+        n += 1
+    return dict(value=tot_f / tot_t / 1e12, unit="TFLOP/s", cores=blas_threads(), kind="oracle",
+                sample=f"{n} of {step.batch} sequences (fixed shuffled order), float64 numpy, "
+                       f"{tot_t:.1f} s")
+
+
 def run_reference(args) -> int:
     world, rank, _ = dist_env()
     if rank != 0:
@@ -516,6 +541,33 @@ def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
         barrier(dev)
     ms_step = max_over_ranks(start.elapsed_time(stop) / args.steps, dev)
     attn_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in evs])), dev)
+
+    # ---------------- end to end: host buffers in, host result out ----------------
+    host = {k: t[k].cpu().pin_memory() for k in ("q", "k_new", "v_new", "slot_mapping",
+                                                 "block_tables", "cu_seqlens_q", "cu_seqlens_k")}
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            for k, v in host.items():
+                t[k].copy_(v, non_blocking=True)
+            one_step()
+            out_host.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+
     peaks = measured_peaks()
     tflops = work["flops"] * world / (ms_step * 1e-3) / 1e12
     attn_tflops = work["flops"] / (attn_ms * 1e-3) / 1e12
@@ -538,7 +590,11 @@ def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
                       traffic=(profile_traffic("prefill_tcgen05_varlen_b32", PREFILL_SOURCES)
                                if args.workload == "prefill_varlen_prefix_hits_b32" else None),
                       peak_source=peaks["source"] + " (MEASURED_PEAKS.json bf16_tflops, burst)"),
+        e2e=dict(value=work["flops"] * world / (e2e_ms * 1e-3) / 1e12, unit="TFLOP/s",
+                 h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=e2e_ms),
         gpu_launches=int(launches), clocks=clocks.summary())
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = prefill_cpu_baseline(step)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
