@@ -19,11 +19,11 @@
 // interleave: while one tile's softmax runs, the tensor core computes the other tile's
 // P V and its next S.  One CTA per SM (persistent; CTA c takes units c, c + grid, ...);
 // the plan kernel lists the pairs, most key tiles first.  Warp roles:
-//   warp 0      TMA producer: Q_A, K_0, Q_B, V_0, then K_j and V_j tiles into a 5-stage
-//               ring (one 3-D tensor-map box per cache block piece; a 128-key tile spans
-//               128 / block_size blocks when the block size is below 128).  Q_B's buffer
-//               frees last (tile B has the most key tiles), so it is loaded after K_0;
-//               the MMA issuer likewise starts S_A0 before waiting for Q_B;
+//   warp 0      TMA producer: K_0, Q_A, V_0, Q_B, then K_j and V_j tiles into a 4-stage
+//               K/V ring (one 3-D tensor-map box per cache block piece; a 128-key tile
+//               spans 128 / block_size blocks when the block size is below 128); the Q
+//               tiles go into a ring of 3 buffers.  The MMA issuer starts S_A0 before
+//               waiting for Q_B;
 //   warp 1      allocates all 512 TMEM columns; one lane issues the MMAs in the order
 //                 S_A0 S_B0 | O_A += P_A0 V_0, S_A1, O_B += P_B0 V_0, S_B1 | ...
 //               where S = Q K_j^T is SS (both operands K-major in shared memory) and
@@ -55,11 +55,13 @@ namespace {
 
 constexpr int kQ = 128;          // query rows per tile (MMA M): tokens x packed heads
 constexpr int kKV = 128;         // keys per tile (MMA N of QK^T, K of PV)
-// K/V ring stages, each one K or one V tile.  A tile takes about 2 us from the TMA issue to
-// its arrival under load, about one key-tile period of a pair, so the producer must run
-// more than a period ahead: with 5 stages V_{j+2} is issued once K_j is consumed.  Five
-// 32 KB stages and the two Q tiles fill the 227 KB of shared memory a CTA may have.
-constexpr int kStages = 5;
+// Shared memory holds seven 32 KB tiles (of the 227 KB a CTA may have): a ring of K/V
+// stages, each one K or one V tile, and a ring of Q tiles.  A tile takes 2 to 5 us from
+// the TMA issue to its arrival under load, and the first tiles of a unit are the ones
+// most often not in L2; with a third Q buffer the next unit's Q_A can be loaded while both
+// Q tiles of the current unit are still in use, which pays more than a fifth K/V stage.
+constexpr int kStages = 4;         // K/V ring stages
+constexpr int kQBufs = 3;          // Q tile ring: tiles A and B of a unit take the next two
 constexpr int kWarps = 12;       // producer, MMA, 2 idle, 2 x 4 softmax
 constexpr int kThreads = kWarps * 32;
 // Register split (setmaxnreg acts on whole warpgroups): the launch gives every thread
@@ -203,11 +205,11 @@ struct Layout {
     static constexpr int REGIONS = D / 64;                  // 64 bf16 = one 128-byte swizzle row
     static constexpr int REGION_BYTES = 128 * 128;          // 128 rows x 128 bytes
     static constexpr int TILE_BYTES = REGIONS * REGION_BYTES;
-    static constexpr int Q_OFF = 0;                         // Q_A, Q_B
-    static constexpr int STAGE_OFF = 2 * TILE_BYTES;
+    static constexpr int Q_OFF = 0;                         // ring of kQBufs Q tiles
+    static constexpr int STAGE_OFF = kQBufs * TILE_BYTES;
     static constexpr int BAR_OFF = STAGE_OFF + kStages * TILE_BYTES;
     // barriers (the per-tile ones come in pairs: + 0 for tile A, + 1 for tile B)
-    static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KVFULL = 4, B_KVEMPTY = B_KVFULL + kStages;
+    static constexpr int B_QFULL = 0, B_QEMPTY = kQBufs, B_KVFULL = 2 * kQBufs, B_KVEMPTY = B_KVFULL + kStages;
     static constexpr int B_SFULL = B_KVEMPTY + kStages, B_PFULL = B_SFULL + 2, B_ODONE = B_PFULL + 2;
     static constexpr int B_OFINAL = B_ODONE + 2, B_OFREE = B_OFINAL + 2, B_DRAIN = B_OFREE + 2;
     static constexpr int B_UFULL = B_DRAIN + 1, B_UEMPTY = B_UFULL + kUnitRing;
@@ -420,13 +422,15 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
 
     if (threadIdx.x == 0) {
         for (int x = 0; x < 2; ++x) {
-            mbar_init(bars + L::B_QFULL + x, 1);
-            mbar_init(bars + L::B_QEMPTY + x, 1);
             mbar_init(bars + L::B_SFULL + x, 1);
             mbar_init(bars + L::B_PFULL + x, 4);
             mbar_init(bars + L::B_ODONE + x, 1);
             mbar_init(bars + L::B_OFINAL + x, 1);
             mbar_init(bars + L::B_OFREE + x, 4);
+        }
+        for (int q = 0; q < kQBufs; ++q) {
+            mbar_init(bars + L::B_QFULL + q, 1);
+            mbar_init(bars + L::B_QEMPTY + q, 1);
         }
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bars + L::B_KVFULL + s, 1);
@@ -498,7 +502,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
         // lane c < 8 holds the physical block of piece c of the next key tile, loaded one
         // key tile ahead so that no copy waits on a block-table lookup.
         uint32_t fill = 0;
-        int qloads[2] = {0, 0};
+        uint32_t qfill = 0;
         const int piece = min(p.block_size, kKV);
         // The block id of piece `lane` of key tile j, or kNoPiece for lanes past the tile's
         // pieces.  The load is only issued here; its value is range-checked where it is
@@ -557,8 +561,9 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             auto load_q = [&](int x) -> bool {
                 const TileInfo& t = x ? tb : ta;
                 if (!t.valid) return true;
-                if (!mbar_wait(bars + L::B_QEMPTY + x, (qloads[x] & 1) ^ 1, abort_flag, p.err)) return false;
-                uint8_t* qdst = smem + L::Q_OFF + x * L::TILE_BYTES;
+                const uint32_t qs = qfill % kQBufs;
+                if (!mbar_wait(bars + L::B_QEMPTY + qs, ((qfill / kQBufs) & 1) ^ 1, abort_flag, p.err)) return false;
+                uint8_t* qdst = smem + L::Q_OFF + qs * L::TILE_BYTES;
                 if constexpr (PREFIX) {
                     // gather the members' query rows into the swizzled Q tile with 16-byte
                     // cp.async copies, all in flight at once: lane l fills rows l, l+32,
@@ -588,16 +593,16 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                     cp_async_wait<0>();
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(bars + L::B_QFULL + x);
+                    if (lane == 0) mbar_arrive(bars + L::B_QFULL + qs);
                 } else {
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(bars + L::B_QFULL + x, L::TILE_BYTES);
+                        mbar_arrive_expect_tx(bars + L::B_QFULL + qs, L::TILE_BYTES);
                         for (int r = 0; r < L::REGIONS; ++r)
-                            tma_load_3d(qdst + r * L::REGION_BYTES, &q_map, bars + L::B_QFULL + x, r * 64,
+                            tma_load_3d(qdst + r * L::REGION_BYTES, &q_map, bars + L::B_QFULL + qs, r * 64,
                                         t.head0, t.q0 + t.tok0);
                     }
                 }
-                ++qloads[x];
+                ++qfill;
                 return true;
             };
             // K (kv = 0) or V tile j, whose block pieces lane c holds in blk_lane; a block id out
@@ -654,10 +659,11 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                        global_ns() - t0 < 100000000ull) {
                 }
             }
-            for (int x = 0; x < 2; ++x) {
-                if (qloads[x] == 0) continue;
+            for (uint32_t q = 0; q < (uint32_t)kQBufs; ++q) {
+                if (qfill <= q) continue;
+                const uint32_t last = qfill - 1 - (qfill - 1 - q) % kQBufs;
                 const uint64_t t0 = global_ns();
-                while (!mbar_try_wait(bars + L::B_QFULL + x, (qloads[x] - 1) & 1) && global_ns() - t0 < 100000000ull) {
+                while (!mbar_try_wait(bars + L::B_QFULL + q, (last / kQBufs) & 1) && global_ns() - t0 < 100000000ull) {
                 }
             }
         }
@@ -670,7 +676,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
         constexpr uint32_t IDESC_QK = idesc_bf16_f32(kQ, kKV, false);
         constexpr uint32_t IDESC_PV = idesc_bf16_f32(kQ, D, true);
         uint32_t fbase = 0;                    // ring fill index of this unit's K_0
-        int quse[2] = {0, 0};                  // Q tiles consumed per slot
+        uint32_t qcons = 0;                    // Q tiles consumed (ring position)
         uint32_t puse[2] = {0, 0};             // P_j waits per tile
         int units[2] = {0, 0};                 // units in which the tile had work
         bool ok = true;
@@ -682,8 +688,8 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
         const uint32_t q_lo = sdesc_sw128_lo(sbase + L::Q_OFF, 16);
         const uint32_t k_lo = sdesc_sw128_lo(sbase + L::STAGE_OFF, 16);
         const uint32_t v_lo = sdesc_sw128_lo(sbase + L::STAGE_OFF, L::REGION_BYTES);
-        auto issue_qk = [&](int x, int kslot) {
-            const uint32_t a = q_lo + (uint32_t)x * TILE16, b = k_lo + (uint32_t)kslot * TILE16;
+        auto issue_qk = [&](int x, int kslot, uint32_t qs) {
+            const uint32_t a = q_lo + qs * TILE16, b = k_lo + (uint32_t)kslot * TILE16;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t o = (kk / 4) * REGION16 + (kk % 4) * 2;   // 64-column region, 32 bytes of K
@@ -714,16 +720,19 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             // S of key tile 0: tile A as soon as Q_A and K_0 are in, then tile B
             if (nkv > 0 && !mbar_wait(bars + L::B_KVFULL + fbase % kStages, (fbase / kStages) & 1, abort_flag, p.err))
                 break;
+            uint32_t qsl[2] = {0, 0};
             for (int x = 0; x < 2 && ok; ++x) {
                 if (!val[x]) continue;
-                if (!mbar_wait(bars + L::B_QFULL + x, quse[x] & 1, abort_flag, p.err)) {
+                qsl[x] = qcons % kQBufs;
+                if (!mbar_wait(bars + L::B_QFULL + qsl[x], (qcons / kQBufs) & 1, abort_flag, p.err)) {
                     ok = false;
                     break;
                 }
+                ++qcons;
                 tc_fence_after();
                 if (lane == 0) {
-                    if (nk[x] > 0) issue_qk(x, fbase % kStages);
-                    if (nk[x] <= 1) umma_commit(bars + L::B_QEMPTY + x);
+                    if (nk[x] > 0) issue_qk(x, fbase % kStages, qsl[x]);
+                    if (nk[x] <= 1) umma_commit(bars + L::B_QEMPTY + qsl[x]);
                 }
                 __syncwarp();
             }
@@ -779,8 +788,8 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                             tc_fence_after();
                         }
                         if (lane == 0) {
-                            issue_qk(x, kslot);
-                            if (j + 2 == nk[x]) umma_commit(bars + L::B_QEMPTY + x);
+                            issue_qk(x, kslot, qsl[x]);
+                            if (j + 2 == nk[x]) umma_commit(bars + L::B_QEMPTY + qsl[x]);
                         }
                         __syncwarp();
                     }
@@ -794,7 +803,6 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             }
             fbase += 2 * (uint32_t)nkv;
             for (int x = 0; x < 2; ++x) {
-                if (val[x]) ++quse[x];
                 if (nk[x] > 0) ++units[x];
             }
         }
