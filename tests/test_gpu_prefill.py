@@ -83,3 +83,60 @@ def test_prefill_last_row_equals_decode(cuda_device):
     torch.cuda.synchronize()
     diff = (out_p[last].float() - out_d.float()).abs().max().item()
     assert diff <= 2e-2
+
+
+def _pack(step):
+    """Query heads per 128-row tile: the GQA group when it is a power of two up to 8."""
+    group = step.num_q_heads // step.num_kv_heads
+    return min(group, 8) if group & (group - 1) == 0 else 1
+
+
+def _expected_pairs(step):
+    """(sequence, tile A, tile B or -1) -> key tiles visited, from the tiling the kernel
+    uses: 128-row query tiles of 128/P tokens x P heads, pairs (2w, 2w + 1) counted from
+    the sequence start, causal bottom-right alignment, 128-key tiles."""
+    tq = 128 // _pack(step)
+    pairs = {}
+    for i in range(step.batch):
+        lq = int(step.cu_seqlens_q[i + 1] - step.cu_seqlens_q[i])
+        lk = int(step.cu_seqlens_k[i + 1] - step.cu_seqlens_k[i])
+        cnt = -(-lq // tq)
+
+        def nkv(qt):
+            tok0, ntok = qt * tq, min(tq, lq - qt * tq)
+            return min(-(-lk // 128), (lk - lq + tok0 + ntok - 1) // 128 + 1)
+
+        for w in range((cnt + 1) // 2):
+            b = 2 * w + 1 if 2 * w + 1 < cnt else -1
+            pairs[(i, 2 * w, b)] = nkv(b if b >= 0 else 2 * w)
+    return pairs
+
+
+@pytest.mark.parametrize("which", ["full", "group4_bs16"])
+def test_prefill_plan_lists_every_pair_longest_first(cuda_device, which):
+    """The plan in the workspace lists each query-tile pair exactly once, sorted by the key
+    tiles it visits, most first (the order inside one count is free)."""
+    if which == "full":
+        step = prefill_varlen_prefix_hits()
+    else:
+        step = make_prefill_step(7, [900, 37, 1, 400, 260], cached_blocks=[10, 0, 0, 3, 16],
+                                 num_q_heads=8, num_kv_heads=2, head_dim=128, block_size=16)
+    t = prefill_to_device(step, cuda_device)
+    ws = torch.zeros(nvpa.varlen_prefill_workspace_size(step.batch, step.total_q), dtype=torch.uint8,
+                     device=cuda_device)
+    nvpa.store_kvcache(t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], t["slot_mapping"])
+    nvpa.varlen_prefill_attention(t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                                  t["cu_seqlens_q"], t["cu_seqlens_k"], step.max_seqlen_q,
+                                  step.max_seqlen_k, step.scale, workspace=ws)
+    torch.cuda.synchronize()
+    head = ws[:8].view(torch.int32).cpu().numpy()
+    n = int(head[0])
+    entries = ws[256:256 + 16 * n].view(torch.int32).cpu().numpy().reshape(n, 4)
+    expected = _expected_pairs(step)
+    got = [(int(e[0]), int(e[1]), int(e[2])) for e in entries]
+    assert sorted(got) == sorted(expected), "the plan must list every pair exactly once"
+    assert all(int(e[3]) == 0 for e in entries)
+    counts = [expected[g] for g in got]
+    assert all(a >= b for a, b in zip(counts, counts[1:])), "pairs must come most key tiles first"
+    # every unit (pair x head group) was claimed: the counter ran at least to the end
+    assert int(head[1]) >= n * (step.num_q_heads // _pack(step))
