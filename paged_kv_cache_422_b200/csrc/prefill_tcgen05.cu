@@ -17,8 +17,8 @@
 // 2w + 1, which has at least as many key tiles; B may be absent).  Both read the same K/V tiles, so
 // each tile is fetched once for 256 query rows, and the two tiles' MMAs and softmaxes
 // interleave: while one tile's softmax runs, the tensor core computes the other tile's
-// P V and its next S.  One CTA per SM (persistent; CTA c takes units c, c + grid, ...);
-// the plan kernel lists the pairs, most key tiles first.  Warp roles:
+// P V and its next S.  One CTA per SM, persistent: the CTAs claim units dynamically from
+// the plan kernel's list, which holds the pairs with the most key tiles first.  Warp roles:
 //   warp 0      TMA producer: K_0, Q_A, V_0, Q_B, then K_j and V_j tiles into a 4-stage
 //               K/V ring (one 3-D tensor-map box per cache block piece; a 128-key tile
 //               spans 128 / block_size blocks when the block size is below 128); the Q
@@ -35,10 +35,10 @@
 // The MMAs of one thread execute in issue order, so S_{j+1} (issued after O += P_j V_j)
 // cannot overwrite P_j early.
 //
-// Stale rows (freed blocks are not cleared, part 1 section 4.3): K rows past the length
-// are masked in the softmax by select (never by arithmetic), and V rows past the length
-// in the last key tile are zeroed in shared memory before their MMAs, so a 0 weight
-// never meets a NaN.
+// Stale rows (freed blocks are not cleared, part 1 section 4.3): the scores of K rows past
+// the length are replaced by -inf with a bit mask (never by arithmetic, which would keep a
+// NaN), and V rows past the length in the last key tile are zeroed in shared memory
+// before their MMAs, so a 0 weight never meets a NaN.
 #include <algorithm>
 #include <climits>
 #include <mutex>
@@ -556,8 +556,8 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             const int32_t* bt = p.block_tables + (size_t)bt_seq * p.max_blocks;
             int cur_blk = load_pieces(bt, ta.kbeg, ta.lk, 0);
             int nxt_blk = nkv > 1 ? load_pieces(bt, ta.kbeg, ta.lk, 1) : kNoPiece;
-            // Q tile x of this unit (its buffer frees after the last S of the previous unit's
-            // tile x)
+            // Q tile x of this unit into the next buffer of the Q ring (a buffer frees after
+            // the last S of the tile that used it, three tiles earlier)
             auto load_q = [&](int x) -> bool {
                 const TileInfo& t = x ? tb : ta;
                 if (!t.valid) return true;
@@ -632,9 +632,10 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                 ++fill;
                 return true;
             };
-            // K_0 first (its ring slot frees early), then Q_A (its buffer frees when the
-            // previous unit's last S of tile A completes), V_0 and Q_B (frees last: tile B has
-            // the most key tiles), then K_j, V_j
+            // K_0 first (its ring slot frees early), then Q_A, V_0, Q_B, then K_j, V_j.  A Q
+            // buffer held the tile three Q loads back: with two tiles per unit, Q_A reuses
+            // tile B's of the unit before last (long done) and Q_B tile A's of the previous
+            // unit (free once that tile's last S completes)
             if (nkv > 0) ok = load_kv(0, 0, cur_blk);
             if (ok) ok = load_q(0);
             if (ok && nkv > 0) ok = load_kv(1, 0, cur_blk);
