@@ -354,7 +354,8 @@ size_t nvpa_varlen_prefill_workspace_size(int batch, int total_q);
  *                   total_q) bytes, 256-byte aligned, no initialisation needed; calls that
  *                   share a workspace must not overlap.
  * A block-table entry outside [0, num_blocks) is flagged (NVPA_FLAG_BAD_BLOCK_ID), its
- * rows are not loaded, and that sequence's output is unspecified (finite).
+ * rows are not read (zeros stand in for them), and that sequence's output is unspecified
+ * but finite.
  * QK^T and PV run on the tensor cores (tcgen05, bf16 inputs, fp32 accumulation in TMEM);
  * P is rounded to bf16 before the PV product.
  * Errors: as for decode.

@@ -616,6 +616,21 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                 const uint32_t valid_mask = __ballot_sync(0xffffffffu, in_range);
                 const uint32_t bytes = (uint32_t)__popc(valid_mask) * (uint32_t)(piece * 128 * L::REGIONS);
                 uint8_t* dst = smem + L::STAGE_OFF + slot * L::TILE_BYTES;
+                // a piece whose block id is out of range is zero-filled instead of loaded (its
+                // keys then score 0 and its values add nothing), so the stage never feeds the
+                // MMAs what a previous tile left there
+                const uint32_t bad_mask = __ballot_sync(0xffffffffu, blk_lane != kNoPiece && !in_range);
+                if (bad_mask != 0) {
+                    for (uint32_t m = bad_mask; m != 0; m &= m - 1) {
+                        const int c = __ffs(m) - 1;
+                        for (int r = 0; r < L::REGIONS; ++r) {
+                            uint4* rows = reinterpret_cast<uint4*>(dst + r * L::REGION_BYTES + c * piece * 128);
+                            for (int k = lane; k < piece * 8; k += 32) rows[k] = make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
                 const CUtensorMap* map = kv ? &v_map : &k_map;
                 if (lane == 0) mbar_arrive_expect_tx(bars + L::B_KVFULL + slot, bytes);
                 for (uint32_t m = valid_mask; m != 0; m &= m - 1) {

@@ -75,3 +75,28 @@ def test_prefill_more_queries_than_keys_is_flagged(cuda_device):
     assert err.item() & nvpa.NVPA_FLAG_BAD_LENGTH
     assert torch.all(out[:50] == 7.0)                 # rows of the bad sequence untouched
     assert torch.isfinite(out[50:].float()).all() and not torch.all(out[50:] == 7.0)
+
+
+def test_prefill_bad_block_id_is_flagged_and_stays_finite(cuda_device):
+    """A block id out of range in one sequence's table is flagged, that piece is not read
+    (zero-filled), the output stays finite, and the other sequences are unaffected."""
+    import oracle
+    from tests.helpers import assert_attention_close, oracle_after_store
+    step = make_prefill_step(5, [300, 140], cached_blocks=[1, 0], num_q_heads=4, num_kv_heads=2,
+                             head_dim=64, block_size=16)
+    t = prefill_to_device(step, cuda_device)
+    nvpa.store_kvcache(t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], t["slot_mapping"])
+    t["block_tables"][0, 3] = step.num_blocks + 7
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    out = nvpa.varlen_prefill_attention(t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                                        t["cu_seqlens_q"], t["cu_seqlens_k"], step.max_seqlen_q,
+                                        step.max_seqlen_k, step.scale, err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() & nvpa.NVPA_FLAG_BAD_BLOCK_ID
+    assert torch.isfinite(out.float()).all()
+    kc, vc, bad = oracle_after_store(step)
+    assert bad == []
+    ref, _ = oracle.varlen_prefill_attention(step.q, kc, vc, step.block_tables, step.cu_seqlens_q,
+                                             step.cu_seqlens_k, step.scale)
+    q1 = int(step.cu_seqlens_q[1])
+    assert_attention_close(out[q1:], ref[q1:], "prefill, sequence with a valid table")
