@@ -115,7 +115,31 @@ def test_prefill_host_checks(lib):
     assert pf(total_q=-3) == _lib.NVPA_ERR_INVALID_ARG
     assert pf(ws=None) == _lib.NVPA_ERR_INVALID_ARG
     assert pf(ws=FAKE + 64) == _lib.NVPA_ERR_INVALID_ARG
-    assert lib.nvpa_varlen_prefill_workspace_size(32, 24594) >= 8 * (32 + 24594 // 128)
+    assert lib.nvpa_varlen_prefill_workspace_size(32, 24594) >= 256 + 16 * (32 + 24594 // 128)
+
+
+def test_prefill_workspace_holds_every_plan_entry(lib):
+    """The prefill plan writes one 16-byte entry per pair of query tiles after a 256-byte
+    header; a tile is 128 / P tokens of one sequence (P = 1, 2, 4 or 8 query heads per
+    tile).  The size query, which sees only the batch and the query rows, must cover the
+    largest pair count any layout of those rows can give."""
+    import numpy as np
+    rng = np.random.default_rng(0)
+    for _ in range(300):
+        batch = int(rng.integers(1, 400))
+        kind = rng.integers(0, 3)
+        if kind == 0:
+            lq = rng.integers(0, 3, size=batch)                 # empty and one-token rows
+        elif kind == 1:
+            lq = rng.choice([1, 15, 16, 17, 31, 33], size=batch)
+        else:
+            lq = rng.integers(0, 5000, size=batch)
+        total_q = int(lq.sum())
+        size = lib.nvpa_varlen_prefill_workspace_size(batch, total_q)
+        for tq in (128, 64, 32, 16):
+            tiles = -(-lq // tq)
+            pairs = int(((tiles + 1) // 2).sum())
+            assert size >= 256 + 16 * pairs, (batch, total_q, tq, pairs, size)
 
 
 def test_gather_host_checks(lib):
