@@ -583,7 +583,9 @@ def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
                     num_q_heads=step.num_q_heads, num_kv_heads=step.num_kv_heads,
                     head_dim=step.head_dim, block_size=step.block_size,
                     algorithmic_tflop=work["flops"] / 1e12,
-                    l2="not flushed: K/V of the step (about 140 MB) is near the 126 MB L2"),
+                    l2="inputs larger than L2, not flushed: each step stores 101 MB of new K/V "
+                       "rows, then reads 101 MB of q and 128 MB of unique K/V and writes 101 MB "
+                       "of output, against the 126 MB L2"),
         roofline=dict(bound="tensor", kernel="varlen_prefill_attention (plan + tcgen05 kernel)",
                       achieved=attn_tflops, peak=peaks["bf16_tflops"], unit="TFLOP/s",
                       frac=attn_tflops / peaks["bf16_tflops"],
