@@ -268,7 +268,10 @@ nvpa_status_t nvpa_decode_step_shared_prefix(
  * nothing (no cudaMalloc, no cudaFree, no allocating library routine).
  *  - The first call on a device resolves the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call before any
- *    stream capture.
+ *    stream capture.  Only a successful resolution is kept: if it fails, the call returns
+ *    NVPA_ERR_CUDA and the next call tries again.  cudaDeviceReset unloads the library's
+ *    device image and makes the kept address stale: do not call this entry point on a
+ *    device again after resetting it in the same process.
  *  - A call whose scratch need (nvpa_paged_decode_workspace_size with the same
  *    arguments) exceeds 64 MiB returns NVPA_ERR_WORKSPACE_TOO_SMALL with a message;
  *    lowering num_splits lowers the need (batch 512 at max_context_len 4096 with 16 query

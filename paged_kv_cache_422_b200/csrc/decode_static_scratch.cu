@@ -12,7 +12,11 @@
 // The array takes kStaticScratchBytes of device memory on every GPU that loads the
 // library, until the process exits.  Its device address is resolved with
 // cudaGetSymbolAddress once per device, during the first call made with that device
-// current; make that first call before any stream capture.  Every call shares the one
+// current; make that first call before any stream capture.  Only a successful resolution
+// is kept: a first call that fails (made during a capture, say) returns the error and the
+// next call tries again.  cudaDeviceReset unloads the library's device image, so an
+// address kept from before a reset is stale: a process that resets a device must not call
+// this entry point on that device again.  Every call shares the one
 // array, and the array keeps the last call's contents: nothing in it has to start at
 // zero (the plan kernel rewrites the counters it needs on every call), but calls whose
 // kernels overlap on the GPU (other streams, other threads) race on it and must be
@@ -29,12 +33,27 @@ constexpr size_t kStaticScratchBytes = size_t(64) << 20;   // 64 MiB
 
 __device__ __align__(256) uint8_t g_decode_scratch[kStaticScratchBytes];
 
+// Per device: the resolved address, or null until a resolution succeeds.
 struct ScratchAddress {
-    std::once_flag once;
+    std::mutex mu;
     void* ptr = nullptr;
-    cudaError_t err = cudaSuccess;
 };
 ScratchAddress g_scratch_address[64];
+
+// The array's device address on the current device `dev`, resolved on first use.
+cudaError_t scratch_address(int dev, void** ptr) {
+    ScratchAddress& sa = g_scratch_address[dev];
+    std::lock_guard<std::mutex> lock(sa.mu);
+    if (sa.ptr == nullptr) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+        if (e != cudaSuccess) return e;
+        if (p == nullptr) return cudaErrorInvalidSymbol;
+        sa.ptr = p;
+    }
+    *ptr = sa.ptr;
+    return cudaSuccess;
+}
 
 }  // namespace
 
@@ -68,14 +87,12 @@ extern "C" nvpa_status_t nvpa_paged_decode_attention_static_scratch(
         set_error("device ordinal %d outside the supported 0..63", dev);
         return NVPA_ERR_UNSUPPORTED;
     }
-    ScratchAddress& sa = g_scratch_address[dev];
-    std::call_once(sa.once, [&] { sa.err = cudaGetSymbolAddress(&sa.ptr, g_decode_scratch); });
-    if (sa.err != cudaSuccess || sa.ptr == nullptr)
-        return cuda_failure(sa.err != cudaSuccess ? sa.err : cudaErrorInvalidSymbol,
-                            "cudaGetSymbolAddress(static decode scratch)");
+    void* scratch = nullptr;
+    e = scratch_address(dev, &scratch);
+    if (e != cudaSuccess) return cuda_failure(e, "cudaGetSymbolAddress(static decode scratch)");
     return nvpa_paged_decode_attention(out, lse_out, q, k_cache, v_cache, block_tables,
                                        max_blocks_per_seq, context_lens, batch, num_q_heads,
                                        num_kv_heads, head_dim, num_blocks, block_size,
-                                       max_context_len, softmax_scale, num_splits, sa.ptr,
+                                       max_context_len, softmax_scale, num_splits, scratch,
                                        kStaticScratchBytes, err_flag, stream);
 }

@@ -4,8 +4,11 @@ It serves callers that cannot allocate device memory (a plugin whose host runtim
 all device memory, or code where an allocation is not allowed).  The test calls it
 through the C ABI twice in a row, on two different problems, and checks each output
 against nvpa_paged_decode_attention with a caller-allocated workspace, within the
-attention tolerance used by every parity test.  The second call also shows that what the
-first call left in the shared scratch array does not leak into the next result.
+attention tolerance used by every parity test, and against the CPU oracle.  The second
+call also shows that what the first call left in the shared scratch array does not leak
+into the next result.  Once both problems have run (so every kernel of the path is
+loaded), repeating both calls must leave the device's free memory unchanged: the entry
+point allocates nothing.
 This file is collected last so that a failure here cannot hide any other test.
 """
 
@@ -17,7 +20,10 @@ import paged_kv_cache_422_b200 as nvpa
 from paged_kv_cache_422_b200 import _lib
 from synth import decode_mid, make_decode_step
 from synth.device import decode_to_device
-from tests.helpers import TOL_ABS, TOL_REL
+from tests.helpers import (TOL_ABS, TOL_REL, assert_attention_close, assert_lse_close,
+                           oracle_after_store)
+
+import oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -43,6 +49,7 @@ def test_static_scratch_matches_workspace_entry_twice(cuda_device):
              make_decode_step(77, [5, 3000, 1, 257, 1800], num_q_heads=32, num_kv_heads=8,
                               head_dim=128, block_size=16)]
     stream = torch.cuda.current_stream(cuda_device)
+    prepared = []
     for step in steps:
         t = decode_to_device(step, cuda_device)
         nvpa.store_kvcache(t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], t["slot_mapping"])
@@ -56,6 +63,24 @@ def test_static_scratch_matches_workspace_entry_twice(cuda_device):
         torch.cuda.synchronize(cuda_device)
         assert _close(out, ref)
         assert np.allclose(lse.cpu().numpy(), ref_lse.cpu().numpy(), atol=2e-3)
+        # and against the oracle itself, on every sequence
+        kc, vc, _ = oracle_after_store(step)
+        ora, ora_lse = oracle.paged_decode_attention(step.q, kc, vc, step.block_tables,
+                                                     step.context_lens, step.scale)
+        assert_attention_close(out, ora, "static scratch decode vs oracle")
+        assert_lse_close(lse, ora_lse, "static scratch decode lse vs oracle")
+        prepared.append((step, t, out, lse, ref))
+
+    # every kernel of both problems is loaded now: repeating both calls allocates nothing
+    torch.cuda.synchronize(cuda_device)
+    free_before, _ = torch.cuda.mem_get_info(cuda_device)
+    for step, t, out, lse, _ in prepared:
+        assert _static_scratch_call(step, t, out, lse, stream) == 0, _lib.lib().nvpa_last_error()
+    torch.cuda.synchronize(cuda_device)
+    free_after, _ = torch.cuda.mem_get_info(cuda_device)
+    assert free_after == free_before, f"device free memory changed by {free_before - free_after} B"
+    for step, t, out, lse, ref in prepared:
+        assert _close(out, ref)
 
 
 def test_static_scratch_rejects_oversized_problem():
