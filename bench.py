@@ -11,6 +11,9 @@ shared prefix is attended once for its group on the tensor cores), nvpa_decode_s
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl nvpa|reference]
                     [--workload NAME]
 
+With --gpus N > 1 and no launcher, bench.py starts N ranks itself (torch.distributed.run
+on 127.0.0.1); under a launcher, N must equal WORLD_SIZE or the run stops with an error.
+
 Prints one JSON line.  `value` is the achieved HBM bandwidth of the whole step in GB/s,
 counting each unique cached K/V row once (plus q, out, the new rows and the index
 arrays); `seq_steps_per_s` is batch / step time.  Under torchrun (N > 1) every rank runs
@@ -209,6 +212,40 @@ def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def launch_plan(gpus: int, env=None):
+    """How this process honours `--gpus N`.
+
+    Returns "run" when the process is one of the job's ranks and the job has N of them,
+    "spawn" when N > 1 and no launcher started the process (bench.py then starts N ranks
+    itself through torch.distributed.run); raises ValueError when a launcher's WORLD_SIZE
+    disagrees with N, so that a run never reports a GPU count it did not use.
+    """
+    env = os.environ if env is None else env
+    if gpus < 1:
+        raise ValueError(f"--gpus must be >= 1, got {gpus}")
+    if "WORLD_SIZE" in env:
+        world = int(env["WORLD_SIZE"])
+        if world != gpus:
+            raise ValueError(f"--gpus {gpus} but the launcher started {world} rank(s) "
+                             f"(WORLD_SIZE={world}); pass matching values")
+        return "run"
+    return "spawn" if gpus > 1 else "run"
+
+
+def spawn_command(gpus: int, argv, port: int):
+    """The torch.distributed.run command line that starts `gpus` ranks of this script."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={gpus}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+            os.path.abspath(__file__)] + list(argv)
+
+
+def _free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
 
 
 def max_over_ranks(value: float, device=None) -> float:
@@ -615,9 +652,17 @@ def main(argv=None) -> int:
     ap.add_argument("--decode-api", choices=["shared", "plain"], default="shared",
                     help="shared: nvpa_decode_step_shared_prefix; plain: nvpa_decode_step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    argv = sys.argv[1:] if argv is None else list(argv)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
+    try:
+        plan = launch_plan(args.gpus)
+    except ValueError as e:
+        print(f"bench.py: {e}", file=sys.stderr, flush=True)
+        return 2
+    if plan == "spawn":
+        return subprocess.call(spawn_command(args.gpus, argv, _free_port()))
     if args.impl == "reference":
         return run_reference(args)
     return run_nvpa(args)

@@ -56,3 +56,34 @@ def test_single_process_helpers_are_identity():
     assert bench.max_over_ranks(3.25) == 3.25
     bench.barrier(None)
     assert bench.dist_env()[0] >= 1
+
+
+def test_gpus_flag_must_match_launcher():
+    import bench
+    assert bench.launch_plan(1, {}) == "run"
+    assert bench.launch_plan(4, {}) == "spawn"
+    assert bench.launch_plan(2, {"WORLD_SIZE": "2"}) == "run"
+    with pytest.raises(ValueError):
+        bench.launch_plan(8, {"WORLD_SIZE": "1"})
+    with pytest.raises(ValueError):
+        bench.launch_plan(1, {"WORLD_SIZE": "4"})
+    with pytest.raises(ValueError):
+        bench.launch_plan(0, {})
+    cmd = bench.spawn_command(4, ["--gpus", "4", "--steps", "3"], 29555)
+    assert cmd[1:4] == ["-m", "torch.distributed.run", "--nnodes=1"]
+    assert "--nproc-per-node=4" in cmd and "127.0.0.1" in cmd and "29555" in cmd
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "3"]
+
+
+def test_mismatched_gpus_flag_fails_loudly():
+    """A --gpus request that disagrees with the launcher's WORLD_SIZE exits non-zero before
+    any GPU work, instead of printing a line with the wrong n_gpus."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "8",
+                        "--steps", "3", "--warmup", "3"], env=env, capture_output=True,
+                       text=True, timeout=120)
+    assert r.returncode != 0
+    assert "--gpus 8" in r.stderr and r.stdout.strip() == ""
