@@ -43,7 +43,14 @@ def _run(step, dev, store=True, num_splits=0, min_group=0, seqs=None):
         step.batch, step.num_q_heads, step.num_kv_heads, step.head_dim, step.max_context_len,
         step.block_size, num_splits, min_group), dtype=torch.uint8, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
-    if store:
+    if store and step.num_tokens > step.batch:
+        # a padded token list (slot -1 entries beyond the batch): the step takes one new
+        # row per sequence, the rows of the real tokens in sequence order
+        real = np.nonzero(step.slot_mapping >= 0)[0][:step.batch]
+        assert len(real) == step.batch
+        sel = torch.as_tensor(real, device=dev)
+        kn, vn, sm = (t[k][sel].contiguous() for k in ("k_new", "v_new", "slot_mapping"))
+    elif store:
         assert step.num_tokens == step.batch
         kn, vn, sm = t["k_new"], t["v_new"], t["slot_mapping"]
     else:
@@ -79,15 +86,26 @@ def _stored(step):
 
 
 def test_batch512_shared_prefix_workload(cuda_device):
+    """The benchmarked step, as bench.py calls it: all 512 sequences against the oracle,
+    both pools bit-exact after the step."""
     step = WORKLOADS["decode_b512_shared_prefix"]()
     shared = np.all(step.block_tables[:, :4] == step.shared_blocks[None, :4], axis=1)
-    seqs = sorted(set(range(0, 512, 17)) | set(np.nonzero(shared)[0][:12].tolist()))
-    (groups, members, tiles), _, _ = _run(step, cuda_device, seqs=seqs)
+    (groups, members, tiles), _, _ = _run(step, cuda_device)
     assert groups == 1
     assert members == int(shared.sum())
     # 1024 prefix keys in 4 partitions of 256; 64 members per query tile (2 query heads
     # each), query tiles in pairs
     assert tiles == 4 * (((members + 63) // 64 + 1) // 2)
+
+
+@pytest.mark.parametrize("name", ["decode_tiny_b4", "decode_mid_b64", "decode_long_b8_ctx32k_bs16"])
+def test_shared_prefix_api_on_the_other_decode_workloads(cuda_device, name):
+    """bench.py times every decode workload through this entry point: the workloads
+    without shared blocks (no group forms, every key goes to the worker), every sequence
+    against the oracle and both pools bit-exact."""
+    step = WORKLOADS[name]()
+    (groups, members, tiles), _, _ = _run(step, cuda_device)
+    assert (groups, members, tiles) == (0, 0, 0)
 
 
 @pytest.mark.parametrize("store", [True, False])
