@@ -404,16 +404,26 @@ SharedGeometry shared_geometry(int batch, int hq, int hkv, int max_context_len, 
 
 }  // namespace
 
-// Keys per decode partition.  Depends on host-side values only.
+// Keys per decode partition.  Depends on host-side values only, so the launch shape and
+// the workspace size are fixed for a given batch and bound (CUDA-graph capturable).
+// Automatic sizing fills the worker's warps: a batch whose contexts all reach
+// max_context_len yields at least kTargetItems work items (one per resident worker warp of
+// a 148-SM B200: 3 CTAs of 4 warps per SM), with partitions of kMinChunkKeys to
+// kMaxChunkKeys keys.  Large batches keep kMaxChunkKeys (fewer partials to merge); small
+// batches with long contexts get more, shorter partitions.
 int decode_chunk_keys(int batch, int num_kv_heads, int max_context_len, int num_splits) {
     const int ctx = std::max(1, max_context_len);
     if (num_splits > 0) {
         const int per = (ctx + num_splits - 1) / num_splits;
         return std::max(kTileKeys, (per + kTileKeys - 1) / kTileKeys * kTileKeys);
     }
-    (void)batch;
-    (void)num_kv_heads;
-    return 256;
+    constexpr long long kTargetItems = 148LL * 3 * kAttnWarps;
+    constexpr int kMinChunkKeys = 64, kMaxChunkKeys = 256;
+    const long long per_partition = (long long)std::max(1, batch) * std::max(1, num_kv_heads);
+    const long long parts = (kTargetItems + per_partition - 1) / per_partition;
+    const long long keys = (ctx + parts - 1) / parts;
+    const long long chunk = (keys + kTileKeys - 1) / kTileKeys * kTileKeys;
+    return (int)std::min<long long>(kMaxChunkKeys, std::max<long long>(kMinChunkKeys, chunk));
 }
 
 size_t decode_workspace_bytes(int batch, int hq, int hkv, int head_dim, int max_context_len,

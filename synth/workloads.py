@@ -448,10 +448,27 @@ def decode_long_fragmented() -> DecodeStep:
                          20000, q_mult=2.0)
 
 
+def decode_graph_batch(batch: int):
+    """Small captured-batch decode shapes (Nano-vLLM part 1, section 5.3 captures decode
+    CUDA graphs for batch 1, 2, 4, 8, 16, ...): `batch` sequences of 4096 tokens (the
+    largest context of the batch-512 workload), 16 query / 8 KV heads, head_dim 128,
+    block size 256, shuffled pool with 16 spare blocks.  Seed 100 + batch.  Used to
+    measure how the split-KV partitioning fills the GPU when the batch is small."""
+    def make() -> DecodeStep:
+        rng = np.random.default_rng(100 + batch)
+        return _build_decode(rng, f"decode_graph_b{batch}_ctx4096", 100 + batch, [4096] * batch,
+                             16, 8, 128, 256, batch * 16 + 16)
+    return make
+
+
 WORKLOADS = {
     "decode_tiny_b4": decode_tiny,
     "decode_mid_b64": decode_mid,
     "decode_b512_shared_prefix": decode_batch512_shared_prefix,
     "prefill_varlen_prefix_hits_b32": prefill_varlen_prefix_hits,
     "decode_long_b8_ctx32k_bs16": decode_long_fragmented,
+    # measurement shapes beyond the five workloads: small captured decode batches
+    "decode_graph_b1_ctx4096": decode_graph_batch(1),
+    "decode_graph_b4_ctx4096": decode_graph_batch(4),
+    "decode_graph_b16_ctx4096": decode_graph_batch(16),
 }

@@ -33,6 +33,17 @@ def _share(step, donor, members, nblocks):
     return step
 
 
+def _prefix_chunk(batch, hkv, max_ctx):
+    """Prefix keys per partition of the shared-prefix step with automatic partitioning:
+    the decode partition (the header's rule: 64 to 256 keys, sized so that a batch of
+    full-length contexts gives about 148 * 3 * 4 work items), rounded up to 128."""
+    per = batch * hkv
+    parts = -(-(148 * 3 * 4) // per)
+    chunk = -(-max_ctx // parts)
+    chunk = min(256, max(64, -(-chunk // 16) * 16))
+    return -(-chunk // 128) * 128
+
+
 def _counters(ws):
     return ws[:20].view(torch.int32).cpu().tolist()[2:5]
 
@@ -129,7 +140,8 @@ def test_shared_prefix_shapes(cuda_device, lens, hq, hkv, d, bs, nshared, nblk, 
     (groups, members, tiles), _, _ = _run(step, cuda_device, store=store, min_group=4)
     assert (groups, members) == (1, nshared)
     tq = 128 // (hq // hkv if (hq // hkv) & (hq // hkv - 1) == 0 else 1)
-    assert tiles == -(-nblk * bs // 256) * ((-(-nshared // tq) + 1) // 2)   # query-tile pairs
+    pchunk = _prefix_chunk(step.batch, hkv, step.max_context_len)
+    assert tiles == -(-nblk * bs // pchunk) * ((-(-nshared // tq) + 1) // 2)   # query-tile pairs
 
 
 def test_two_groups_and_a_short_common_run(cuda_device):
@@ -143,7 +155,9 @@ def test_two_groups_and_a_short_common_run(cuda_device):
     step.block_tables[19, 2:4] = step.block_tables[20, 2:4]   # 19: common run of 2
     (groups, members, tiles), _, _ = _run(step, cuda_device, min_group=4)
     assert (groups, members) == (2, 20)
-    assert tiles == 1 + 1      # one query tile (pair) and one partition each (160 and 64 keys)
+    # one query tile (pair) per group; prefixes of 160 and 64 keys in partitions of pchunk
+    pchunk = _prefix_chunk(step.batch, 2, step.max_context_len)
+    assert tiles == -(-160 // pchunk) + -(-64 // pchunk)
 
 
 def test_member_whose_private_part_is_its_new_token(cuda_device):
