@@ -79,8 +79,9 @@ typedef enum nvpa_status {
                                      [0, num_blocks): its rows are treated as absent        */
 #define NVPA_FLAG_BAD_LENGTH   4  /* a context length / cumulative length outside the bounds
                                      declared by the call: clamped to those bounds          */
-#define NVPA_FLAG_TIMEOUT      8  /* a tensor-core kernel's internal wait exceeded its time
-                                     limit (2 s): the kernel stopped early, outputs are
+#define NVPA_FLAG_TIMEOUT      8  /* a tensor-core kernel stopped early: an internal wait
+                                     exceeded its time limit (2 s), or its shared memory
+                                     did not start 1024-byte aligned; outputs are
                                      incomplete; never expected in correct operation        */
 
 /* Library version, as 10000*major + 100*minor + patch. */
@@ -153,7 +154,10 @@ size_t nvpa_paged_decode_workspace_size(int batch, int num_q_heads, int num_kv_h
  *   context_lens    int32 [batch], each in [0, max_context_len] and at most
  *                   max_blocks_per_seq * block_size (else clamped, NVPA_FLAG_BAD_LENGTH).
  *   max_context_len host-side upper bound of context_lens (sizes the partitioning).
- *   num_splits      0 = automatic; n > 0 = cut the longest possible context into at
+ *   num_splits      0 = automatic: partitions of 64 to 256 keys, sized from batch,
+ *                   num_kv_heads and max_context_len so that a batch of full-length
+ *                   contexts gives about 1776 work items (one per resident worker warp
+ *                   of a 148-SM B200); n > 0 = cut the longest possible context into at
  *                   most n partitions (rounded to the library's tile size).
  *   workspace       device scratch of at least nvpa_paged_decode_workspace_size(...)
  *                   bytes, 256-byte aligned; contents need no initialisation and are

@@ -40,7 +40,9 @@
 // NaN), and V rows past the length in the last key tile are zeroed in shared memory
 // before their MMAs, so a 0 weight never meets a NaN.
 #include <algorithm>
+#include <cfloat>
 #include <climits>
+#include <cmath>
 #include <mutex>
 
 #include "attn_warp.cuh"
@@ -106,18 +108,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // cache with two softmax warps, and the fully unrolled row loops are most of the kernel's
 // code.
 
-// x = s * scale (log2 units) in place, two scores per packed multiply.
-__device__ __forceinline__ void scale_row(uint32_t (&sv)[kKV], float sc) {
-    const uint64_t sc2 = f2_pack(sc, sc);
-#pragma unroll
-    for (int k = 0; k < kKV; k += 2) {
-        float a, b;
-        f2_unpack(f2_mul(f2_pack(__uint_as_float(sv[k]), __uint_as_float(sv[k + 1])), sc2), a, b);
-        sv[k] = __float_as_uint(a);
-        sv[k + 1] = __float_as_uint(b);
-    }
-}
-
 // Columns at or past lim - key0 (keys the row does not see, including rows past the
 // sequence) become -inf by bit mask, whatever they held.
 __device__ __forceinline__ void mask_row(uint32_t (&sv)[kKV], int key0, int lim) {
@@ -141,19 +131,21 @@ __device__ __forceinline__ float row_max(const uint32_t (&sv)[kKV]) {
     return fmaxf(e0, e1);
 }
 
-// P = exp2(x + nm) of one row, packed to bf16 pairs and written over the first kKV/2 TMEM
+// P = exp2(s * c + nm) of one row of raw scores (c > 0: the scale in log2 units; one packed
+// FMA per pair of scores), packed to bf16 pairs and written over the first kKV/2 TMEM
 // columns of the row (32 S columns become 16 P columns, each chunk's P landing in columns
-// already read); returns the row sum of the fp32 values.  A -inf x gives 0.
-__device__ __forceinline__ float exp_row(const uint32_t (&sv)[kKV], uint32_t s_col, float nm) {
-    const uint64_t nm2 = f2_pack(nm, nm);
+// already read); returns the row sum of the fp32 values.  A -inf score or offset gives 0.
+__device__ __forceinline__ float exp_row(const uint32_t (&sv)[kKV], uint32_t s_col, float c, float nm) {
+    const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(nm, nm);
     uint64_t l0 = f2_pack(0.f, 0.f), l1 = l0;
 #pragma unroll
-    for (int c = 0; c < kKV / 32; ++c) {
+    for (int cc = 0; cc < kKV / 32; ++cc) {
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 32; k += 2) {
             float a, b;
-            f2_unpack(f2_add(f2_pack(__uint_as_float(sv[c * 32 + k]), __uint_as_float(sv[c * 32 + k + 1])), nm2), a, b);
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[cc * 32 + k]), __uint_as_float(sv[cc * 32 + k + 1])), c2, nm2),
+                      a, b);
             a = fast_exp2(a);
             b = fast_exp2(b);
             const uint64_t p2 = f2_pack(a, b);
@@ -163,12 +155,20 @@ __device__ __forceinline__ float exp_row(const uint32_t (&sv)[kKV], uint32_t s_c
                 l0 = f2_add(l0, p2);
             pk[k / 2] = pack_bf16x2(a, b);
         }
-        tmem_st16(s_col + c * 16, pk);
+        tmem_st16(s_col + cc * 16, pk);
     }
     float a0, b0, a1, b1;
     f2_unpack(l0, a0, b0);
     f2_unpack(l1, a1, b1);
     return (a0 + b0) + (a1 + b1);
+}
+
+// One 32-byte global store (the address must be 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8]) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                 :: "l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]),
+                    "r"(w[7])
+                 : "memory");
 }
 
 struct PrefillParams {
@@ -197,7 +197,9 @@ struct PrefillParams {
     int hgroups;                 // head groups, hq / P
     int max_blocks, num_blocks, block_size, block_shift;
     int max_q, max_k, causal;
-    float scale_log2;
+    float scale_log2;            // |scale| * log2(e) (a negative scale flips the sign of Q K^T)
+    int negate_qk;               // scale < 0: S = -Q K^T
+    int out_v8;                  // out is 32-byte aligned: 32-byte stores in the epilogue
 };
 
 template <int D>
@@ -689,7 +691,9 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
         // O_B += P_Bj V_j, S_B(j+1).  Tile A's softmax of key tile j+1 thus overlaps tile
         // B's P V and S MMAs, and the other way round.  K_j's ring slot is released after
         // the last S that reads it, V_j's after the last P V.
-        constexpr uint32_t IDESC_QK = idesc_bf16_f32(kQ, kKV, false);
+        // a negative softmax scale is applied as S = -Q K^T (the descriptor's negate-A bit),
+        // so the softmax always multiplies by a positive factor
+        const uint32_t IDESC_QK = idesc_bf16_f32(kQ, kKV, false) | (p.negate_qk ? (1u << 13) : 0u);
         constexpr uint32_t IDESC_PV = idesc_bf16_f32(kQ, D, true);
         uint32_t fbase = 0;                    // ring fill index of this unit's K_0
         uint32_t qcons = 0;                    // Q tiles consumed (ring position)
@@ -874,11 +878,10 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                 for (int c = 0; c < kKV / 32; ++c)
                     tmem_ld32(s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
                 tmem_wait_ld();
-                // scaled scores, keys the row does not see at -inf (diagonal tiles only),
-                // then the row's largest value
-                scale_row(sv, p.scale_log2);
+                // keys the row does not see at -inf (diagonal tiles only), then the row's
+                // largest value in log2 units (raw scores times a positive factor)
                 if (!open) mask_row(sv, key0, lim);
-                const float mt = row_max(sv);
+                const float mt = row_max(sv) * p.scale_log2;
                 const bool over = mt > m + kRescaleSlack;
                 const bool rescale = __any_sync(0xffffffffu, over);
                 float alpha = 1.f;
@@ -888,9 +891,10 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                     l *= alpha;
                     m = m_new;
                 }
-                // P_j = exp2(x - m) as bf16 pairs over the first kKV/2 columns of S_j.  A row
-                // with no visible key yet (m = -inf) gets exp2(-inf) = 0 through its offset.
-                l += exp_row(sv, s_col, m > -INFINITY ? -m : -INFINITY);
+                // P_j = exp2(s * scale - m) as bf16 pairs over the first kKV/2 columns of S_j.
+                // A row with no visible key yet (m = -inf) gets exp2(-inf) = 0 through its
+                // offset.
+                l += exp_row(sv, s_col, p.scale_log2, m > -INFINITY ? -m : -INFINITY);
                 if (rescale && j > 0) {
                     // O holds P_0..P_{j-1} V (all complete once S_j is): rescale it before
                     // P_j is released to the MMA
@@ -945,6 +949,19 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                         __stcg(reinterpret_cast<float4*>(pdst + c * 32 + 4 * q),
                                make_float4(__uint_as_float(o[4 * q + 0]) * inv, __uint_as_float(o[4 * q + 1]) * inv,
                                            __uint_as_float(o[4 * q + 2]) * inv, __uint_as_float(o[4 * q + 3]) * inv));
+                } else if (row_ok && p.out_v8) {
+                    // 32-byte stores: each fills a whole sector of the output row (a warp's
+                    // 32 rows are 32 different lines, so the count of store instructions is
+                    // what the epilogue's time goes by)
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        uint32_t w[8];
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            w[k] = pack_bf16x2(__uint_as_float(o[16 * q + 2 * k]) * inv,
+                                               __uint_as_float(o[16 * q + 2 * k + 1]) * inv);
+                        st_global_v8(dst + c * 4 + 2 * q, w);
+                    }
                 } else if (row_ok) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
@@ -978,6 +995,16 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
 // ------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------
+// The softmax scale in log2 units.  The kernel multiplies raw scores by a positive factor
+// (one packed FMA together with the max subtraction); a negative scale flips the sign of
+// Q K^T in the MMA instead, and a zero scale becomes the smallest normal float (every score
+// then rounds to 0, the weights are uniform, and a masked -inf score still weighs 0).
+void set_scale(PrefillParams& p, float scale) {
+    const float a = std::fabs(scale) * kLog2e;
+    p.scale_log2 = a > 0.f ? a : FLT_MIN;
+    p.negate_qk = scale < 0.f;
+}
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -1014,12 +1041,23 @@ template <int D, bool PREFIX>
 cudaError_t launch_prefill(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
                            const PrefillParams& p, int grid, cudaStream_t stream, bool pdl = PREFIX) {
     static std::once_flag once[64];
+    static int launch_regs[64];
     int dev = 0;
     cudaGetDevice(&dev);
-    std::call_once(once[dev & 63], [] {
+    std::call_once(once[dev & 63], [dev] {
         cudaFuncSetAttribute(prefill_tcgen05_kernel<D, PREFIX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Layout<D>::ALLOC);
+        cudaFuncAttributes fa{};
+        launch_regs[dev & 63] =
+            cudaFuncGetAttributes(&fa, prefill_tcgen05_kernel<D, PREFIX>) == cudaSuccess ? fa.numRegs : 0;
     });
+    // The warpgroups' setmaxnreg shares add up to kLaunchRegs per thread: with fewer registers
+    // at launch the raising warpgroups could never get their share, so do not launch.
+    if (launch_regs[dev & 63] != kLaunchRegs) {
+        set_error("prefill kernel compiled with %d registers per thread, %d expected", launch_regs[dev & 63],
+                  kLaunchRegs);
+        return cudaErrorInvalidConfiguration;
+    }
     if (!pdl) {
         prefill_tcgen05_kernel<D, PREFIX><<<grid, kThreads, Layout<D>::ALLOC, stream>>>(qm, km, vm, p);
         return cudaGetLastError();
@@ -1080,7 +1118,7 @@ cudaError_t launch_decode_prefix_tcgen05(const DecodePrefixArgs& a, cudaStream_t
     p.num_blocks = a.num_blocks;
     p.block_size = a.block_size;
     p.block_shift = __builtin_ctz((unsigned)a.block_size);
-    p.scale_log2 = a.scale * kLog2e;
+    set_scale(p, a.scale);
     const long long units = std::max(1LL, a.max_entries) * p.hgroups * 2;   // single-tile units
     const long long cap = a.max_ctas > 0 ? a.max_ctas : (long long)device_sm_count();
     const int grid = (int)std::max(1LL, std::min<long long>(cap, units));
@@ -1140,7 +1178,8 @@ nvpa_status_t run_varlen_prefill_tcgen05(const PrefillCall& c, void* workspace, 
     p.max_q = c.max_seqlen_q;
     p.max_k = c.max_seqlen_k;
     p.causal = c.causal;
-    p.scale_log2 = c.scale * kLog2e;
+    set_scale(p, c.scale);
+    p.out_v8 = (reinterpret_cast<uintptr_t>(c.out) & 31u) == 0;
 
     prefill_plan_kernel<<<1, 1024, 0, stream>>>(p, reinterpret_cast<int4*>(ws + 256), reinterpret_cast<int32_t*>(ws));
     cudaError_t e = cudaGetLastError();

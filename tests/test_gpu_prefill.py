@@ -68,6 +68,21 @@ def test_prefill_small_shapes(cuda_device, lens, cached, hq, hkv, d, bs, causal)
     assert_lse_close(lse, ora_lse, f"prefill {lens} causal={causal}")
 
 
+@pytest.mark.parametrize("scale", [-0.125, 0.0, 0.6])
+def test_prefill_scale_sign_and_size(cuda_device, scale):
+    """A negative softmax scale (the kernel flips the sign of Q K^T on the tensor cores and
+    scales by its magnitude), a zero scale (uniform weights over the visible keys) and a
+    large one (sharp rows whose running maximum moves often)."""
+    step = make_prefill_step(55, [700, 300, 129], cached_blocks=[1, 0, 0], num_q_heads=8,
+                             num_kv_heads=2, head_dim=128, block_size=64, scale=scale)
+    assert step.scale == scale
+    t = prefill_to_device(step, cuda_device)
+    out, lse = _run(step, t)
+    ora_out, ora_lse = _oracle(step)
+    assert_attention_close(out, ora_out, f"prefill scale {scale}")
+    assert_lse_close(lse, ora_lse, f"prefill scale {scale}")
+
+
 def test_prefill_last_row_equals_decode(cuda_device):
     """The last query row of a causal prefill sees the whole context: decode of the same
     token over the same cache gives the same attention."""
