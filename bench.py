@@ -301,31 +301,71 @@ def prepare_oracle(step):
     step._ora_k, step._ora_v = kc, vc
 
 
-def cpu_baseline(step, budget_s: float = 12.0) -> dict:
-    """The oracle on as many whole sequences (in a fixed shuffled order) as fit in about
-    budget_s seconds; GB/s counts each sampled sequence's K/V bytes."""
-    prepare_oracle(step)
+def effective_cores(cpu_s: float, wall_s: float) -> int:
+    """Host cores a run kept busy on average: process CPU time (all threads) / wall time."""
+    return max(1, int(round(cpu_s / wall_s))) if wall_s > 0 else 1
+
+
+def single_thread():
+    """Context that limits the BLAS pools to one thread (the 1-thread CPU baseline)."""
+    from threadpoolctl import threadpool_limits
+    return threadpool_limits(limits=1)
+
+
+def _decode_cpu_run(step, budget_s):
     order = np.random.default_rng(0).permutation(step.batch)
     tot_t, tot_b, n = 0.0, 0, 0
+    c0, w0 = time.process_time(), time.perf_counter()
     while n < step.batch and tot_t < budget_s:
         dt, nb = oracle_decode_sample(step, order[n:n + 4])
         tot_t += dt
         tot_b += nb
         n += len(order[n:n + 4])
-    return dict(value=tot_b / tot_t / 1e9, unit="GB/s", cores=blas_threads(), kind="oracle",
+    cores = effective_cores(time.process_time() - c0, time.perf_counter() - w0)
+    return tot_t, tot_b, n, cores
+
+
+def cpu_baseline(step, budget_s: float = 8.0) -> dict:
+    """The oracle on as many whole sequences (in a fixed shuffled order) as fit in about
+    budget_s seconds, with the host's BLAS threads and again with one thread; GB/s counts
+    each sampled sequence's K/V bytes.  `cores` is the average number of host cores the
+    run kept busy (process CPU time / wall time), not the size of the thread pool."""
+    prepare_oracle(step)
+    tot_t, tot_b, n, cores = _decode_cpu_run(step, budget_s)
+    with single_thread():
+        t1, b1, n1, _ = _decode_cpu_run(step, budget_s)
+    return dict(value=tot_b / tot_t / 1e9, unit="GB/s", cores=cores, kind="oracle",
+                blas_threads=blas_threads(),
                 sample=f"{n} of {step.batch} sequences (fixed shuffled order), float64 numpy, "
-                       f"{tot_t:.1f} s; seq-steps/s {n / tot_t:.3f}")
+                       f"{tot_t:.1f} s; seq-steps/s {n / tot_t:.3f}",
+                single_thread=dict(value=b1 / t1 / 1e9, unit="GB/s", cores=1,
+                                   sample=f"{n1} sequences, {t1:.1f} s, BLAS limited to 1 thread"))
 
 
-def prefill_cpu_baseline(step, budget_s: float = 10.0) -> dict:
+def prefill_cpu_baseline(step, budget_s: float = 8.0) -> dict:
     """The oracle's varlen prefill on as many whole sequences (in a fixed shuffled order) as
-    fit in about budget_s seconds; TFLOP/s counts the sample's algorithmic causal FLOPs."""
+    fit in about budget_s seconds, with the host's BLAS threads and again with one thread;
+    TFLOP/s counts the sample's algorithmic causal FLOPs.  `cores` as in cpu_baseline."""
     import oracle
     kc, vc = step.k_pool.copy(), step.v_pool.copy()
     oracle.store_kvcache(kc, vc, step.k_new, step.v_new, step.slot_mapping)
+    tot_t, tot_f, n, cores = _prefill_cpu_run(step, kc, vc, budget_s)
+    with single_thread():
+        t1, f1, n1, _ = _prefill_cpu_run(step, kc, vc, budget_s)
+    return dict(value=tot_f / tot_t / 1e12, unit="TFLOP/s", cores=cores, kind="oracle",
+                blas_threads=blas_threads(),
+                sample=f"{n} of {step.batch} sequences (fixed shuffled order), float64 numpy, "
+                       f"{tot_t:.1f} s",
+                single_thread=dict(value=f1 / t1 / 1e12, unit="TFLOP/s", cores=1,
+                                   sample=f"{n1} sequences, {t1:.1f} s, BLAS limited to 1 thread"))
+
+
+def _prefill_cpu_run(step, kc, vc, budget_s):
+    import oracle
     d, hq = step.head_dim, step.num_q_heads
     order = np.random.default_rng(0).permutation(step.batch)
     tot_t, tot_f, n = 0.0, 0, 0
+    c0, w0 = time.process_time(), time.perf_counter()
     while n < step.batch and tot_t < budget_s:
         i = int(order[n])
         q0, q1 = int(step.cu_seqlens_q[i]), int(step.cu_seqlens_q[i + 1])
@@ -337,9 +377,7 @@ def prefill_cpu_baseline(step, budget_s: float = 10.0) -> dict:
         tot_t += time.perf_counter() - t0
         tot_f += 4 * d * hq * (lq * (lk - lq) + lq * (lq + 1) // 2)
         n += 1
-    return dict(value=tot_f / tot_t / 1e12, unit="TFLOP/s", cores=blas_threads(), kind="oracle",
-                sample=f"{n} of {step.batch} sequences (fixed shuffled order), float64 numpy, "
-                       f"{tot_t:.1f} s")
+    return tot_t, tot_f, n, effective_cores(time.process_time() - c0, time.perf_counter() - w0)
 
 
 def run_reference(args) -> int:
@@ -352,15 +390,18 @@ def run_reference(args) -> int:
     order = np.random.default_rng(0).permutation(step.batch)
     per_step = 4
     times, nbytes = [], []
+    cpu_used = 0.0
     for i in range(args.warmup + args.steps):
         seqs = order[(i * per_step) % step.batch:][:per_step]
+        c0 = time.process_time()
         dt, nb = oracle_decode_sample(step, seqs)
         if i >= args.warmup:
             times.append(dt)
             nbytes.append(nb)
+            cpu_used += time.process_time() - c0
     t = float(np.sum(times))
     value = float(np.sum(nbytes)) / t / 1e9
-    cores = blas_threads()
+    cores = effective_cores(cpu_used, t)
     line = dict(metric=METRIC, value=value, unit="GB/s", n_gpus=args.gpus, steps=args.steps,
                 warmup=args.warmup, ms_per_step=t / args.steps * 1e3, higher_is_better=True,
                 scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
@@ -376,6 +417,121 @@ def run_reference(args) -> int:
 # ----------------------------------------------------------------------------------
 # the GPU arm
 # ----------------------------------------------------------------------------------
+
+def make_l2_flush(dev, enabled: bool):
+    """A function that evicts the 126 MB L2 by writing a 512 MB buffer on `stream` (between
+    timed steps, outside their events), or None when flushing is off."""
+    if not enabled:
+        return None
+    import torch
+    buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    def flush(stream):
+        with torch.cuda.stream(stream):
+            buf.fill_(1)
+    return flush
+
+
+class PackedInputs:
+    """A step's input tensors laid out back to back (256-byte aligned) in one pinned host
+    buffer and in one device buffer of the same layout, so that a single cudaMemcpyAsync
+    moves all of a step's inputs; `views` are device tensors with the original shapes and
+    dtypes inside the device buffer."""
+
+    def __init__(self, tensors: dict, dev):
+        import torch
+        offs, off = {}, 0
+        for k, v in tensors.items():
+            nb = v.numel() * v.element_size()
+            offs[k] = (off, nb)
+            off = (off + nb + 255) // 256 * 256
+        self.host = torch.empty(off, dtype=torch.uint8).pin_memory()
+        self.device = torch.empty(off, dtype=torch.uint8, device=dev)
+        self.views = {}
+        for k, v in tensors.items():
+            o, nb = offs[k]
+            self.host[o:o + nb].copy_(v.detach().contiguous().reshape(-1).view(torch.uint8).cpu())
+            self.views[k] = self.device[o:o + nb].view(v.dtype).view(v.shape)
+        self.nbytes = off
+
+    def upload(self, stream):
+        import torch
+        with torch.cuda.stream(stream):
+            self.device.copy_(self.host, non_blocking=True)
+
+
+def end_to_end(run_step, packed, out, stream, steps, warmup, dev):
+    """Steps with host inputs and a host result, all inside the timed region: one packed
+    host-to-device copy of the step's inputs, the step on the device copies, and the output
+    copied back to pinned host memory.  The read-back of step i runs on a second stream
+    while step i + 1's inputs upload; step i + 1's kernels wait for it (they overwrite
+    `out`), and the timed region ends after the last read-back.  Returns (ms per step,
+    breakdown of medians: h2d, compute, d2h in device ms and host ms spent enqueueing a
+    step, d2h bytes per step)."""
+    import torch
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    copy_stream = torch.cuda.Stream(device=dev)
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(5)]   # noqa: E731
+
+    def one(ev, prev):
+        ev[0].record(stream)
+        packed.upload(stream)
+        ev[1].record(stream)
+        if prev is not None:
+            stream.wait_event(prev[4])          # the previous read-back is done with `out`
+        run_step(packed.views)
+        ev[2].record(stream)
+        copy_stream.wait_event(ev[2])
+        ev[3].record(copy_stream)
+        with torch.cuda.stream(copy_stream):
+            out_host.copy_(out, non_blocking=True)
+        ev[4].record(copy_stream)
+
+    prev = None
+    for _ in range(max(1, warmup)):
+        ev = mk()
+        one(ev, prev)
+        prev = ev
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    evs = [mk() for _ in range(steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    host_s = []
+    e0.record(stream)
+    prev = None
+    for i in range(steps):
+        h0 = time.perf_counter()
+        one(evs[i], prev)
+        host_s.append(time.perf_counter() - h0)
+        prev = evs[i]
+    stream.wait_event(prev[4])
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    br = dict(h2d_ms=float(np.median([e[0].elapsed_time(e[1]) for e in evs])),
+              compute_ms=float(np.median([e[1].elapsed_time(e[2]) for e in evs])),
+              d2h_ms=float(np.median([e[3].elapsed_time(e[4]) for e in evs])),
+              host_enqueue_ms=float(np.median(host_s)) * 1e3)
+    return ms, br, out_host.numel() * out_host.element_size()
+
+
+def timed_steps(step_fn, steps, stream, flush, dev):
+    """Run `steps` steps on `stream`, each bracketed by CUDA events; with `flush`, L2 is
+    evicted before every step, outside its events.  Returns (total ms of the region, list of
+    per-step ms); the caller takes the step time from the events when flushing."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        if flush is not None:
+            flush(stream)
+        step_fn(evs[i])
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    return start.elapsed_time(stop), [a.elapsed_time(b) for a, b in evs]
+
 
 def run_nvpa(args) -> int:
     import torch
@@ -420,12 +576,13 @@ def run_nvpa(args) -> int:
     out = torch.empty_like(t["q"])
     decode_call = nvpa.decode_step_shared_prefix if shared else nvpa.decode_step
 
-    def one_step(ev=None):
+    def one_step(ev=None, inp=None):
         # store + decode in one call (the library's fused decode step)
+        inp = t if inp is None else inp
         if ev is not None:
             ev[0].record(stream)
-        decode_call(t["q"], t["k_new"], t["v_new"], t["k_cache"], t["v_cache"],
-                    t["slot_mapping"], t["block_tables"], t["context_lens"],
+        decode_call(inp["q"], inp["k_new"], inp["v_new"], t["k_cache"], t["v_cache"],
+                    inp["slot_mapping"], inp["block_tables"], inp["context_lens"],
                     step.max_context_len, step.scale, out=out, workspace=workspace,
                     num_splits=args.num_splits, stream=stream)
         if ev is not None:
@@ -437,51 +594,28 @@ def run_nvpa(args) -> int:
     torch.cuda.synchronize(dev)
 
     # ---------------- timed region: K steps, device-timed ----------------
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush = make_l2_flush(dev, args.flush_l2)
     with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
         barrier(dev)
         torch.cuda.synchronize(dev)
         n0 = lib.nvpa_kernel_launch_count()
-        start.record(stream)
-        for i in range(args.steps):
-            one_step(evs[i])
-        stop.record(stream)
-        torch.cuda.synchronize(dev)
+        ms_total, per_step = timed_steps(one_step, args.steps, stream, flush, dev)
         launches = lib.nvpa_kernel_launch_count() - n0
         barrier(dev)
-    ms_total = start.elapsed_time(stop)
-    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    if flush is not None:
+        ms_total = float(np.sum(per_step))     # the flushes between steps are not step time
+    attn_ms = max_over_ranks(float(np.mean(per_step)), dev)
+    median_ms = max_over_ranks(float(np.median(per_step)), dev)
     ms_total = max_over_ranks(ms_total, dev)
-    attn_ms = max_over_ranks(attn_ms, dev)
     ms_step = ms_total / args.steps
 
     # ---------------- end to end: host buffers in, host result out ----------------
-    host = {k: t[k].cpu().pin_memory() for k in ("q", "k_new", "v_new", "slot_mapping",
-                                                 "block_tables", "context_lens")}
-    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = out_host.numel() * out_host.element_size()
-
-    def e2e_step():
-        with torch.cuda.stream(stream):
-            for k, v in host.items():
-                t[k].copy_(v, non_blocking=True)
-            one_step()
-            out_host.copy_(out, non_blocking=True)
-
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
-    torch.cuda.synchronize(dev)
-    barrier(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    packed = PackedInputs({k: t[k] for k in ("q", "k_new", "v_new", "slot_mapping",
+                                             "block_tables", "context_lens")}, dev)
+    e2e_ms, e2e_breakdown, d2h = end_to_end(lambda inp: one_step(inp=inp), packed, out, stream,
+                                            args.steps, args.warmup, dev)
+    e2e_ms = max_over_ranks(e2e_ms, dev)
+    h2d = packed.nbytes
 
     peaks = measured_peaks()
     value = work["step"] * world / (ms_step * 1e-3) / 1e9
@@ -495,6 +629,7 @@ def run_nvpa(args) -> int:
         metric=METRIC, value=value, unit="GB/s", n_gpus=world, steps=args.steps,
         warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",
         vs_baseline=None, dtype="bf16", data="synthetic",
+        ms_per_step_median=median_ms,
         pct_of_peak=100.0 * value / world / peaks["hbm_gbs"],
         seq_steps_per_s=step.batch * world / (ms_step * 1e-3),
         logical_kv_gbs=work["kv_logical"] * world / (ms_step * 1e-3) / 1e9,
@@ -504,8 +639,13 @@ def run_nvpa(args) -> int:
                     total_context_tokens=int(step.context_lens.sum()),
                     unique_kv_bytes=work["kv_unique"], step_bytes=work["step"],
                     parallelism=f"replicas x{world}" if world > 1 else "single GPU",
-                    l2="inputs larger than L2: %.2f GB of unique K/V per step vs 126 MB L2"
-                       % (work["kv_unique"] / 1e9),
+                    l2=("flushed: a 512 MB write before every step, outside its events; "
+                        "%.3f GB of unique K/V per step vs 126 MB L2" % (work["kv_unique"] / 1e9))
+                       if args.flush_l2 else
+                       ("inputs larger than L2: %.2f GB of unique K/V per step vs 126 MB L2"
+                        % (work["kv_unique"] / 1e9) if work["kv_unique"] > L2_BYTES else
+                        "NOT flushed (--flush-l2 flushes): %.3f GB of unique K/V per step fits "
+                        "in the 126 MB L2" % (work["kv_unique"] / 1e9)),
                     num_splits=args.num_splits,
                     decode_api=("nvpa_decode_step_shared_prefix" if shared else "nvpa_decode_step")),
         roofline=dict(bound="hbm",
@@ -516,7 +656,11 @@ def run_nvpa(args) -> int:
                       frac=attn_gbs / peaks["hbm_gbs"], traffic=traffic,
                       peak_source=peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, burst copy)"),
         e2e=dict(value=work["step"] * world / (e2e_ms * 1e-3) / 1e9, unit="GB/s",
-                 h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=e2e_ms),
+                 h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=e2e_ms,
+                 copies="one packed host-to-device copy of the step's inputs on the step's "
+                        "stream; the read-back of out on a copy stream, overlapping the next "
+                        "step's upload; all inside the timed region",
+                 breakdown_median=e2e_breakdown),
         gpu_launches=int(launches),
         clocks=cs,
     )
@@ -546,13 +690,14 @@ def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
                      dtype=torch.uint8, device=dev)
     out = torch.empty_like(t["q"])
 
-    def one_step(ev=None):
-        nvpa.store_kvcache(t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], t["slot_mapping"],
-                           stream=stream)
+    def one_step(ev=None, inp=None):
+        inp = t if inp is None else inp
+        nvpa.store_kvcache(inp["k_new"], inp["v_new"], t["k_cache"], t["v_cache"],
+                           inp["slot_mapping"], stream=stream)
         if ev is not None:
             ev[0].record(stream)
-        nvpa.varlen_prefill_attention(t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
-                                      t["cu_seqlens_q"], t["cu_seqlens_k"], step.max_seqlen_q,
+        nvpa.varlen_prefill_attention(inp["q"], t["k_cache"], t["v_cache"], inp["block_tables"],
+                                      inp["cu_seqlens_q"], inp["cu_seqlens_k"], step.max_seqlen_q,
                                       step.max_seqlen_k, step.scale, out=out, workspace=ws,
                                       stream=stream)
         if ev is not None:
@@ -562,48 +707,40 @@ def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
         for _ in range(args.warmup):
             one_step()
     torch.cuda.synchronize(dev)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush = make_l2_flush(dev, args.flush_l2)
+
+    step_evs = []
+
+    def timed_whole(ev):
+        a = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        one_step(ev)
+        b = torch.cuda.Event(enable_timing=True)
+        b.record(stream)
+        step_evs.append((a, b))
+
     with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
         barrier(dev)
         torch.cuda.synchronize(dev)
         n0 = lib.nvpa_kernel_launch_count()
-        start.record(stream)
-        for i in range(args.steps):
-            one_step(evs[i])
-        stop.record(stream)
-        torch.cuda.synchronize(dev)
+        ms_total, attn_per_step = timed_steps(timed_whole, args.steps, stream, flush, dev)
         launches = lib.nvpa_kernel_launch_count() - n0
         barrier(dev)
-    ms_step = max_over_ranks(start.elapsed_time(stop) / args.steps, dev)
-    attn_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in evs])), dev)
+    whole = [a.elapsed_time(b) for a, b in step_evs]
+    if flush is not None:
+        ms_total = float(np.sum(whole))
+    ms_step = max_over_ranks(ms_total / args.steps, dev)
+    attn_ms = max_over_ranks(float(np.mean(attn_per_step)), dev)
+    attn_median_ms = max_over_ranks(float(np.median(attn_per_step)), dev)
+    median_ms = max_over_ranks(float(np.median(whole)), dev)
 
     # ---------------- end to end: host buffers in, host result out ----------------
-    host = {k: t[k].cpu().pin_memory() for k in ("q", "k_new", "v_new", "slot_mapping",
-                                                 "block_tables", "cu_seqlens_q", "cu_seqlens_k")}
-    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = out_host.numel() * out_host.element_size()
-
-    def e2e_step():
-        with torch.cuda.stream(stream):
-            for k, v in host.items():
-                t[k].copy_(v, non_blocking=True)
-            one_step()
-            out_host.copy_(out, non_blocking=True)
-
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
-    torch.cuda.synchronize(dev)
-    barrier(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    packed = PackedInputs({k: t[k] for k in ("q", "k_new", "v_new", "slot_mapping",
+                                             "block_tables", "cu_seqlens_q", "cu_seqlens_k")}, dev)
+    e2e_ms, e2e_breakdown, d2h = end_to_end(lambda inp: one_step(inp=inp), packed, out, stream,
+                                            args.steps, args.warmup, dev)
+    e2e_ms = max_over_ranks(e2e_ms, dev)
+    h2d = packed.nbytes
 
     peaks = measured_peaks()
     tflops = work["flops"] * world / (ms_step * 1e-3) / 1e12
@@ -613,6 +750,7 @@ def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
         value=tflops, unit="TFLOP/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
         ms_per_step=ms_step, higher_is_better=True, scaling="weak", vs_baseline=None,
         dtype="bf16", data="synthetic",
+        ms_per_step_median=median_ms, attention_ms_median=attn_median_ms,
         tokens_per_s=step.total_q * world / (ms_step * 1e-3),
         store_gbs=work["store"] / ((ms_step - attn_ms) * 1e-3) / 1e9 if ms_step > attn_ms else None,
         config=dict(workload=args.workload, batch=step.batch, total_q=step.total_q,
@@ -620,9 +758,11 @@ def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
                     num_q_heads=step.num_q_heads, num_kv_heads=step.num_kv_heads,
                     head_dim=step.head_dim, block_size=step.block_size,
                     algorithmic_tflop=work["flops"] / 1e12,
-                    l2="inputs larger than L2, not flushed: each step stores 101 MB of new K/V "
-                       "rows, then reads 101 MB of q and 128 MB of unique K/V and writes 101 MB "
-                       "of output, against the 126 MB L2"),
+                    l2=("flushed: a 512 MB write before every step, outside its events"
+                        if args.flush_l2 else
+                        "inputs larger than L2, not flushed: each step stores 101 MB of new K/V "
+                        "rows, then reads 101 MB of q and 128 MB of unique K/V and writes 101 MB "
+                        "of output, against the 126 MB L2")),
         roofline=dict(bound="tensor", kernel="varlen_prefill_attention (plan + tcgen05 kernel)",
                       achieved=attn_tflops, peak=peaks["bf16_tflops"], unit="TFLOP/s",
                       frac=attn_tflops / peaks["bf16_tflops"],
@@ -630,7 +770,11 @@ def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
                                if args.workload == "prefill_varlen_prefix_hits_b32" else None),
                       peak_source=peaks["source"] + " (MEASURED_PEAKS.json bf16_tflops, burst)"),
         e2e=dict(value=work["flops"] * world / (e2e_ms * 1e-3) / 1e12, unit="TFLOP/s",
-                 h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=e2e_ms),
+                 h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=e2e_ms,
+                 copies="one packed host-to-device copy of the step's inputs on the step's "
+                        "stream; the read-back of out on a copy stream, overlapping the next "
+                        "step's upload; all inside the timed region",
+                 breakdown_median=e2e_breakdown),
         gpu_launches=int(launches), clocks=clocks.summary())
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = prefill_cpu_baseline(step)
@@ -652,6 +796,8 @@ def main(argv=None) -> int:
     ap.add_argument("--decode-api", choices=["shared", "plain"], default="shared",
                     help="shared: nvpa_decode_step_shared_prefix; plain: nvpa_decode_step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--flush-l2", action="store_true",
+                    help="write a 512 MB buffer before every timed step (outside its events)")
     argv = sys.argv[1:] if argv is None else list(argv)
     args = ap.parse_args(argv)
     if args.warmup < 3:
