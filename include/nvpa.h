@@ -80,9 +80,8 @@ typedef enum nvpa_status {
 #define NVPA_FLAG_BAD_LENGTH   4  /* a context length / cumulative length outside the bounds
                                      declared by the call: clamped to those bounds          */
 #define NVPA_FLAG_TIMEOUT      8  /* a tensor-core kernel stopped early: an internal wait
-                                     exceeded its time limit (2 s), or its shared memory
-                                     did not start 1024-byte aligned; outputs are
-                                     incomplete; never expected in correct operation        */
+                                     exceeded its time limit (2 s); outputs are incomplete;
+                                     never expected in correct operation                    */
 
 /* Library version, as 10000*major + 100*minor + patch. */
 int nvpa_version(void);
@@ -154,11 +153,13 @@ size_t nvpa_paged_decode_workspace_size(int batch, int num_q_heads, int num_kv_h
  *   context_lens    int32 [batch], each in [0, max_context_len] and at most
  *                   max_blocks_per_seq * block_size (else clamped, NVPA_FLAG_BAD_LENGTH).
  *   max_context_len host-side upper bound of context_lens (sizes the partitioning).
- *   num_splits      0 = automatic: partitions of 64 to 256 keys, sized from batch,
- *                   num_kv_heads and max_context_len so that a batch of full-length
- *                   contexts gives about 1776 work items (one per resident worker warp
- *                   of a 148-SM B200); n > 0 = cut the longest possible context into at
- *                   most n partitions (rounded to the library's tile size).
+ *   num_splits      0 = automatic: partitions sized from batch, num_kv_heads and
+ *                   max_context_len (counting full-length contexts) against the 1776
+ *                   resident worker warps of a 148-SM B200: small batches get at least
+ *                   one item per warp (partitions of 64 keys or more), many sequences
+ *                   256-key partitions, a few long sequences about two rounds of items
+ *                   (128 to 1024 keys); n > 0 = cut the longest possible context into
+ *                   at most n partitions (rounded to the library's tile size).
  *   workspace       device scratch of at least nvpa_paged_decode_workspace_size(...)
  *                   bytes, 256-byte aligned; contents need no initialisation and are
  *                   overwritten.  Calls that share a workspace must not overlap.

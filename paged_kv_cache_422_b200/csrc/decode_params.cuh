@@ -71,6 +71,41 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 
 
+// Worker items are ordered by length, longest first, in this many classes of a partition's
+// key count (class c holds lengths with c = length * 256 / chunk).
+constexpr int kLengthClasses = 256;
+__device__ __forceinline__ int length_class(int len, int chunk) {
+    return min(kLengthClasses - 1, (int)(((long long)len * kLengthClasses) / chunk));
+}
+
+// Exclusive prefix sum of v over the block (every thread calls it; blockDim a multiple of
+// 32, at most 1024); total = the block's sum.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& total) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    if (lane == 31) warp_tot[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+        int w = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += n;
+        }
+        warp_tot[lane] = w;
+    }
+    __syncthreads();
+    const int excl = incl - v + (wid ? warp_tot[wid - 1] : 0);
+    total = warp_tot[31];
+    __syncthreads();
+    return excl;
+}
+
 constexpr int kSharedTable = 2 * kSharedMaxBatch;   // buckets of the shared-prefix plan (a power of two)
 constexpr size_t kSharedPlanSmem = sizeof(int) * (6 * (size_t)kSharedTable + 2 * (size_t)kSharedMaxBatch);
 

@@ -23,32 +23,6 @@ namespace nvpa {
 // [3] members, [4] prefix work units (pairs of query tiles of one group and partition),
 // [5] the prefix kernel's unit counter.
 
-__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& total) {
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
-    }
-    if (lane == 31) warp_tot[wid] = incl;
-    __syncthreads();
-    if (wid == 0) {
-        int w = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xffffffffu, w, o);
-            if (lane >= o) w += n;
-        }
-        warp_tot[lane] = w;
-    }
-    __syncthreads();
-    const int excl = incl - v + (wid ? warp_tot[wid - 1] : 0);
-    total = warp_tot[31];
-    __syncthreads();
-    return excl;
-}
-
 __global__ void __launch_bounds__(1024) decode_plan_shared_kernel(const AttnParams p) {
     extern __shared__ int sh[];
     int* tkey = sh;                            // first block id of the bucket, -1 = empty
@@ -190,22 +164,51 @@ __global__ void __launch_bounds__(1024) decode_plan_shared_kernel(const AttnPara
     __syncthreads();
 
     // 5. worker items for the private partitions
+    // Every full-length partition first, sequence by sequence, then each sequence's last,
+    // shorter partition, longest first (a counting sort over 256 length classes): the
+    // items claimed last are the shortest, so the worker's warps finish close together.
+    __shared__ int s_cls[kLengthClasses];
+    for (int i = tid; i < kLengthClasses; i += blockDim.x) s_cls[i] = 0;
+    __syncthreads();
     int carry = 0;
     for (int base = 0; base < p.batch; base += blockDim.x) {
         const int b = base + tid;
-        int nsp = 0, npc = 0, pre = 0, ctx = 0;
+        int nfull = 0, npc = 0, nsp = 0, pre = 0;
         if (b < p.batch) {
             pre = s_slot[b];
-            ctx = s_ctx[b];
+            const int priv = s_ctx[b] - pre;
             npc = (pre + p.pchunk - 1) / p.pchunk;
-            nsp = max(1, (ctx - pre + p.chunk - 1) / p.chunk);
+            nsp = max(1, (priv + p.chunk - 1) / p.chunk);
+            const int last = priv - (nsp - 1) * p.chunk;
+            nfull = last == p.chunk ? nsp : nsp - 1;
+            if (last < p.chunk) atomicAdd(s_cls + length_class(last, p.chunk), 1);
         }
         int block_tot = 0;
-        const int e = carry + block_exclusive_scan(nsp, warp_tot, block_tot);
-        for (int s = 0; s < nsp; ++s)
-            p.items[e + s] = make_int4(b, (npc + s) | ((npc + nsp) << 16), pre + s * p.chunk,
-                                       min(ctx, pre + (s + 1) * p.chunk));
+        const int e = carry + block_exclusive_scan(nfull, warp_tot, block_tot);
+        for (int s = 0; s < nfull; ++s)
+            p.items[e + s] = make_int4(b, (npc + s) | ((npc + nsp) << 16), pre + s * p.chunk, pre + (s + 1) * p.chunk);
         carry += block_tot;
+    }
+    __syncthreads();
+    // first position of each length class, longest class first, after the full partitions
+    {
+        const int cls = kLengthClasses - 1 - tid;
+        const int v = tid < kLengthClasses ? s_cls[cls] : 0;
+        int tot_short = 0;
+        const int e = block_exclusive_scan(v, warp_tot, tot_short);
+        if (tid < kLengthClasses) s_cls[cls] = carry + e;
+        __syncthreads();
+        for (int b = tid; b < p.batch; b += blockDim.x) {
+            const int pre = s_slot[b], ctx = s_ctx[b];
+            const int priv = ctx - pre;
+            const int npc = (pre + p.pchunk - 1) / p.pchunk;
+            const int nsp = max(1, (priv + p.chunk - 1) / p.chunk);
+            const int last = priv - (nsp - 1) * p.chunk;
+            if (last == p.chunk) continue;
+            const int pos = atomicAdd(s_cls + length_class(last, p.chunk), 1);
+            p.items[pos] = make_int4(b, (npc + nsp - 1) | ((npc + nsp) << 16), pre + (nsp - 1) * p.chunk, ctx);
+        }
+        carry += tot_short;
     }
     if (tid == 0) {
         p.counter[0] = 0;

@@ -30,55 +30,63 @@ namespace nvpa {
 // plan: context lengths -> (sequence, partition, key range) table
 // ------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) decode_plan_kernel(const AttnParams p) {
+    // Items: every full-length partition first, sequence by sequence, then each sequence's
+    // last, shorter partition, longest first (a counting sort over kLengthClasses length
+    // classes): the items claimed last are the shortest, so the worker's warps finish
+    // close together.
     __shared__ int warp_tot[32];
-    __shared__ int carry_s;
+    __shared__ int s_cls[kLengthClasses];
     const int tid = threadIdx.x;
     pdl_launch_dependents();
-    const int lane = tid & 31, wid = tid >> 5;
-    if (tid == 0) carry_s = 0;
+    for (int i = tid; i < kLengthClasses; i += blockDim.x) s_cls[i] = 0;
     __syncthreads();
     const long long lim_ll = min((long long)p.max_ctx, (long long)p.max_blocks * p.block_size);
     const int lim = (int)lim_ll;
-    for (int base = 0; base < p.batch; base += 1024) {
+    auto clamp_ctx = [&](int b, bool flag) {
+        int ctx = __ldg(p.context_lens + b);
+        if (ctx < 0 || ctx > lim) {
+            if (flag) flag_error(p.err, NVPA_FLAG_BAD_LENGTH);
+            ctx = min(max(ctx, 0), lim);
+        }
+        return ctx;
+    };
+    int carry = 0;
+    for (int base = 0; base < p.batch; base += blockDim.x) {
         const int b = base + tid;
-        int ns = 0, ctx = 0;
+        int nfull = 0, ns = 0;
         if (b < p.batch) {
-            ctx = __ldg(p.context_lens + b);
-            if (ctx < 0 || ctx > lim) {
-                flag_error(p.err, NVPA_FLAG_BAD_LENGTH);
-                ctx = min(max(ctx, 0), lim);
-            }
+            const int ctx = clamp_ctx(b, true);
             ns = max(1, (ctx + p.chunk - 1) / p.chunk);
             p.nsplit[b] = ns;
+            const int last = ctx - (ns - 1) * p.chunk;
+            nfull = last == p.chunk ? ns : ns - 1;
+            if (last < p.chunk) atomicAdd(s_cls + length_class(last, p.chunk), 1);
         }
-        int v = ns;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            int n = __shfl_up_sync(0xffffffffu, v, o);
-            if (lane >= o) v += n;
-        }
-        if (lane == 31) warp_tot[wid] = v;
-        __syncthreads();
-        if (wid == 0) {
-            int w = warp_tot[lane];
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                int n = __shfl_up_sync(0xffffffffu, w, o);
-                if (lane >= o) w += n;
-            }
-            warp_tot[lane] = w;
-        }
-        __syncthreads();
-        const int excl = carry_s + (v - ns) + (wid ? warp_tot[wid - 1] : 0);
-        for (int s = 0; s < ns; ++s)
-            p.items[excl + s] = make_int4(b, s | (ns << 16), s * p.chunk, min(ctx, (s + 1) * p.chunk));
-        __syncthreads();
-        if (tid == 1023) carry_s = excl + ns;
-        __syncthreads();
+        int block_tot = 0;
+        const int e = carry + block_exclusive_scan(nfull, warp_tot, block_tot);
+        for (int s = 0; s < nfull; ++s)
+            p.items[e + s] = make_int4(b, s | (ns << 16), s * p.chunk, (s + 1) * p.chunk);
+        carry += block_tot;
+    }
+    __syncthreads();
+    // first position of each length class, longest class first, after the full partitions
+    const int cls = kLengthClasses - 1 - tid;
+    const int v = tid < kLengthClasses ? s_cls[cls] : 0;
+    int tot_short = 0;
+    const int e = block_exclusive_scan(v, warp_tot, tot_short);
+    if (tid < kLengthClasses) s_cls[cls] = carry + e;
+    __syncthreads();
+    for (int b = tid; b < p.batch; b += blockDim.x) {
+        const int ctx = clamp_ctx(b, false);
+        const int ns = max(1, (ctx + p.chunk - 1) / p.chunk);
+        const int last = ctx - (ns - 1) * p.chunk;
+        if (last == p.chunk) continue;
+        const int pos = atomicAdd(s_cls + length_class(last, p.chunk), 1);
+        p.items[pos] = make_int4(b, (ns - 1) | (ns << 16), (ns - 1) * p.chunk, ctx);
     }
     if (tid == 0) {
         p.counter[0] = 0;
-        p.counter[1] = carry_s * p.hkv;
+        p.counter[1] = (carry + tot_short) * p.hkv;
         p.counter[2] = p.counter[3] = p.counter[4] = 0;   // no shared-prefix groups
     }
 }
@@ -406,11 +414,16 @@ SharedGeometry shared_geometry(int batch, int hq, int hkv, int max_context_len, 
 
 // Keys per decode partition.  Depends on host-side values only, so the launch shape and
 // the workspace size are fixed for a given batch and bound (CUDA-graph capturable).
-// Automatic sizing fills the worker's warps: a batch whose contexts all reach
-// max_context_len yields at least kTargetItems work items (one per resident worker warp of
-// a 148-SM B200: 3 CTAs of 4 warps per SM), with partitions of kMinChunkKeys to
-// kMaxChunkKeys keys.  Large batches keep kMaxChunkKeys (fewer partials to merge); small
-// batches with long contexts get more, shorter partitions.
+// Automatic sizing counts a batch of full-length contexts against kTargetItems, the
+// resident worker warps of a 148-SM B200 (3 CTAs of 4 warps per SM):
+//  - small batches get partitions of 64 keys or more, enough for one item per warp;
+//  - many sequences (more than kTargetItems / 8 sequence-head pairs) keep 256-key
+//    partitions: their lengths vary, and the rounds of items even out by themselves;
+//  - a few long sequences get about two rounds of items, 128 to 1024 keys each: fewer,
+//    longer partitions mean fewer partials to write and merge, and two rounds keep the
+//    warps that idle in the last one a small share (measured on 8 contexts of 32 k keys:
+//    592-key partitions beat 256-key ones by 6 %, 240-key ones lost 6 %; on 16 contexts of
+//    4 k keys 160-key partitions beat 256-key ones by 12 %).
 int decode_chunk_keys(int batch, int num_kv_heads, int max_context_len, int num_splits) {
     const int ctx = std::max(1, max_context_len);
     if (num_splits > 0) {
@@ -418,12 +431,16 @@ int decode_chunk_keys(int batch, int num_kv_heads, int max_context_len, int num_
         return std::max(kTileKeys, (per + kTileKeys - 1) / kTileKeys * kTileKeys);
     }
     constexpr long long kTargetItems = 148LL * 3 * kAttnWarps;
-    constexpr int kMinChunkKeys = 64, kMaxChunkKeys = 256;
+    constexpr long long kMinChunkKeys = 64, kMaxChunkKeys = 256, kMinLongChunk = 128, kMaxLongChunk = 1024;
+    auto round16 = [](long long k) { return (k + kTileKeys - 1) / kTileKeys * kTileKeys; };
     const long long per_partition = (long long)std::max(1, batch) * std::max(1, num_kv_heads);
-    const long long parts = (kTargetItems + per_partition - 1) / per_partition;
-    const long long keys = (ctx + parts - 1) / parts;
-    const long long chunk = (keys + kTileKeys - 1) / kTileKeys * kTileKeys;
-    return (int)std::min<long long>(kMaxChunkKeys, std::max<long long>(kMinChunkKeys, chunk));
+    const long long fill = round16((ctx + (kTargetItems + per_partition - 1) / per_partition - 1) /
+                                   ((kTargetItems + per_partition - 1) / per_partition));
+    if (fill < kMaxChunkKeys) return (int)std::max(kMinChunkKeys, fill);
+    if (per_partition * 8 > kTargetItems) return (int)kMaxChunkKeys;
+    const long long parts = (2 * kTargetItems + per_partition - 1) / per_partition;
+    const long long chunk = round16((ctx + parts - 1) / parts);
+    return (int)std::min(kMaxLongChunk, std::max(kMinLongChunk, chunk));
 }
 
 size_t decode_workspace_bytes(int batch, int hq, int hkv, int head_dim, int max_context_len,
