@@ -107,6 +107,14 @@ def measured_peaks() -> dict:
                     bf16_tflops_sustained=1400.0, source="fallback")
 
 
+def peak_source(peaks: dict, key: str, what: str) -> str:
+    """Where a roofline denominator came from, for the JSON line."""
+    if peaks["source"] == "measured":
+        return f"measured: MEASURED_PEAKS.json {key} ({what})"
+    return (f"fallback: MEASURED_PEAKS.json absent; an earlier measurement of the same "
+            f"quantity ({what}) on this kind of B200: {peaks[key]:g}")
+
+
 class ClockSampler:
     """nvidia-smi clock/throttle samples taken while the timed region runs."""
 
@@ -654,7 +662,7 @@ def run_nvpa(args) -> int:
                               "decode step: plan, split-KV worker with the store folded in, combine"),
                       achieved=attn_gbs, peak=peaks["hbm_gbs"], unit="GB/s",
                       frac=attn_gbs / peaks["hbm_gbs"], traffic=traffic,
-                      peak_source=peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, burst copy)"),
+                      peak_source=peak_source(peaks, "hbm_gbs", "burst copy")),
         e2e=dict(value=work["step"] * world / (e2e_ms * 1e-3) / 1e9, unit="GB/s",
                  h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=e2e_ms,
                  copies="one packed host-to-device copy of the step's inputs on the step's "
@@ -768,7 +776,7 @@ def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
                       frac=attn_tflops / peaks["bf16_tflops"],
                       traffic=(profile_traffic("prefill_tcgen05_varlen_b32", PREFILL_SOURCES)
                                if args.workload == "prefill_varlen_prefix_hits_b32" else None),
-                      peak_source=peaks["source"] + " (MEASURED_PEAKS.json bf16_tflops, burst)"),
+                      peak_source=peak_source(peaks, "bf16_tflops", "cuBLAS bf16 GEMM, burst")),
         e2e=dict(value=work["flops"] * world / (e2e_ms * 1e-3) / 1e12, unit="TFLOP/s",
                  h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=e2e_ms,
                  copies="one packed host-to-device copy of the step's inputs on the step's "
