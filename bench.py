@@ -426,17 +426,26 @@ def run_reference(args) -> int:
 # the GPU arm
 # ----------------------------------------------------------------------------------
 
+L2_FLUSHED = "flushed: a 512 MB buffer written and read back before every step, outside its events"
+
+
 def make_l2_flush(dev, enabled: bool):
-    """A function that evicts the 126 MB L2 by writing a 512 MB buffer on `stream` (between
-    timed steps, outside their events), or None when flushing is off."""
+    """A function that evicts the 126 MB L2 on `stream` (between timed steps, outside their
+    events), or None when flushing is off: it writes a 512 MB buffer, then reads it back,
+    so that L2 ends up holding clean lines of that buffer; after the write alone L2 would
+    be full of dirty lines, and the next step would pay for writing them back to DRAM
+    inside its own events."""
     if not enabled:
         return None
     import torch
     buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    words = buf.view(torch.int32)
+    res = torch.empty((), dtype=torch.int32, device=dev)
 
     def flush(stream):
         with torch.cuda.stream(stream):
             buf.fill_(1)
+            torch.amax(words, dim=0, out=res)
     return flush
 
 
@@ -467,58 +476,89 @@ class PackedInputs:
         with torch.cuda.stream(stream):
             self.device.copy_(self.host, non_blocking=True)
 
+    def twin(self) -> "PackedInputs":
+        """A second device buffer of the same layout, filled from the same host buffer."""
+        import torch
+        t = object.__new__(PackedInputs)
+        t.host, t.nbytes = self.host, self.nbytes
+        t.device = torch.empty_like(self.device)
+        base = self.device.data_ptr()
+        t.views = {}
+        for k, v in self.views.items():
+            o = v.data_ptr() - base
+            nb = v.numel() * v.element_size()
+            t.views[k] = t.device[o:o + nb].view(v.dtype).view(v.shape)
+        return t
+
+
+E2E_COPIES = ("every step: one packed host-to-device copy of all its inputs from pinned memory and "
+              "a device-to-host copy of its output, both inside the timed region; double-buffered "
+              "so that step i+1's upload and step i-1's read-back overlap step i's kernels")
+
 
 def end_to_end(run_step, packed, out, stream, steps, warmup, dev):
-    """Steps with host inputs and a host result, all inside the timed region: one packed
-    host-to-device copy of the step's inputs, the step on the device copies, and the output
-    copied back to pinned host memory.  The read-back of step i runs on a second stream
-    while step i + 1's inputs upload; step i + 1's kernels wait for it (they overwrite
-    `out`), and the timed region ends after the last read-back.  Returns (ms per step,
-    breakdown of medians: h2d, compute, d2h in device ms and host ms spent enqueueing a
-    step, d2h bytes per step)."""
+    """Steps with host inputs and a host result, all inside the timed region: every step
+    copies all of its inputs from pinned host memory (one packed host-to-device copy),
+    runs on the device copies, and copies its output back to pinned host memory.
+    Consecutive steps are independent batches, so the copies are pipelined the way a
+    serving loop prefetches: two device input buffers and two output buffers, uploads on
+    one stream, kernels on `stream`, read-backs on a third; step i + 1's upload and step
+    i - 1's read-back run while step i computes.  A buffer is reused only after the step
+    that used it two steps earlier is done with it.  The timed region starts before the
+    first upload and ends after the last read-back.  `run_step(inputs, out)` enqueues one
+    step on `stream`.  Returns (ms per step, breakdown of medians: h2d, compute, d2h in
+    device ms and host ms spent enqueueing a step, d2h bytes per step)."""
     import torch
+    packs = [packed, packed.twin()]
+    outs = [out, torch.empty_like(out)]
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    copy_stream = torch.cuda.Stream(device=dev)
-    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(5)]   # noqa: E731
+    up = torch.cuda.Stream(device=dev)
+    down = torch.cuda.Stream(device=dev)
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(6)]   # noqa: E731
 
-    def one(ev, prev):
-        ev[0].record(stream)
-        packed.upload(stream)
-        ev[1].record(stream)
-        if prev is not None:
-            stream.wait_event(prev[4])          # the previous read-back is done with `out`
-        run_step(packed.views)
+    # ev: 0/1 upload start/end (up), 2/3 compute start/end (stream), 4/5 read-back (down)
+    def one(i, ev, hist):
+        b = i & 1
+        if i >= 2:
+            up.wait_event(hist[i - 2][3])       # step i - 2 has finished reading this input buffer
+        ev[0].record(up)
+        packs[b].upload(up)
+        ev[1].record(up)
+        stream.wait_event(ev[1])
+        if i >= 2:
+            stream.wait_event(hist[i - 2][5])   # step i - 2's read-back is done with this output
         ev[2].record(stream)
-        copy_stream.wait_event(ev[2])
-        ev[3].record(copy_stream)
-        with torch.cuda.stream(copy_stream):
-            out_host.copy_(out, non_blocking=True)
-        ev[4].record(copy_stream)
+        run_step(packs[b].views, outs[b])
+        ev[3].record(stream)
+        down.wait_event(ev[3])
+        ev[4].record(down)
+        with torch.cuda.stream(down):
+            out_host.copy_(outs[b], non_blocking=True)
+        ev[5].record(down)
 
-    prev = None
-    for _ in range(max(1, warmup)):
-        ev = mk()
-        one(ev, prev)
-        prev = ev
+    hist = []
+    for i in range(max(2, warmup)):
+        hist.append(mk())
+        one(i, hist[-1], hist)
     torch.cuda.synchronize(dev)
     barrier(dev)
-    evs = [mk() for _ in range(steps)]
+    hist = []
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    host_s = []
     e0.record(stream)
-    prev = None
+    up.wait_event(e0)
+    host_s = []
     for i in range(steps):
         h0 = time.perf_counter()
-        one(evs[i], prev)
+        hist.append(mk())
+        one(i, hist[-1], hist)
         host_s.append(time.perf_counter() - h0)
-        prev = evs[i]
-    stream.wait_event(prev[4])
+    stream.wait_event(hist[-1][5])
     e1.record(stream)
     torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1) / steps
-    br = dict(h2d_ms=float(np.median([e[0].elapsed_time(e[1]) for e in evs])),
-              compute_ms=float(np.median([e[1].elapsed_time(e[2]) for e in evs])),
-              d2h_ms=float(np.median([e[3].elapsed_time(e[4]) for e in evs])),
+    br = dict(h2d_ms=float(np.median([e[0].elapsed_time(e[1]) for e in hist])),
+              compute_ms=float(np.median([e[2].elapsed_time(e[3]) for e in hist])),
+              d2h_ms=float(np.median([e[4].elapsed_time(e[5]) for e in hist])),
               host_enqueue_ms=float(np.median(host_s)) * 1e3)
     return ms, br, out_host.numel() * out_host.element_size()
 
@@ -584,15 +624,15 @@ def run_nvpa(args) -> int:
     out = torch.empty_like(t["q"])
     decode_call = nvpa.decode_step_shared_prefix if shared else nvpa.decode_step
 
-    def one_step(ev=None, inp=None):
+    def one_step(ev=None, inp=None, dst=None):
         # store + decode in one call (the library's fused decode step)
         inp = t if inp is None else inp
         if ev is not None:
             ev[0].record(stream)
         decode_call(inp["q"], inp["k_new"], inp["v_new"], t["k_cache"], t["v_cache"],
                     inp["slot_mapping"], inp["block_tables"], inp["context_lens"],
-                    step.max_context_len, step.scale, out=out, workspace=workspace,
-                    num_splits=args.num_splits, stream=stream)
+                    step.max_context_len, step.scale, out=out if dst is None else dst,
+                    workspace=workspace, num_splits=args.num_splits, stream=stream)
         if ev is not None:
             ev[1].record(stream)
 
@@ -620,8 +660,8 @@ def run_nvpa(args) -> int:
     # ---------------- end to end: host buffers in, host result out ----------------
     packed = PackedInputs({k: t[k] for k in ("q", "k_new", "v_new", "slot_mapping",
                                              "block_tables", "context_lens")}, dev)
-    e2e_ms, e2e_breakdown, d2h = end_to_end(lambda inp: one_step(inp=inp), packed, out, stream,
-                                            args.steps, args.warmup, dev)
+    e2e_ms, e2e_breakdown, d2h = end_to_end(lambda inp, o: one_step(inp=inp, dst=o), packed, out,
+                                            stream, args.steps, args.warmup, dev)
     e2e_ms = max_over_ranks(e2e_ms, dev)
     h2d = packed.nbytes
 
@@ -647,8 +687,8 @@ def run_nvpa(args) -> int:
                     total_context_tokens=int(step.context_lens.sum()),
                     unique_kv_bytes=work["kv_unique"], step_bytes=work["step"],
                     parallelism=f"replicas x{world}" if world > 1 else "single GPU",
-                    l2=("flushed: a 512 MB write before every step, outside its events; "
-                        "%.3f GB of unique K/V per step vs 126 MB L2" % (work["kv_unique"] / 1e9))
+                    l2=(L2_FLUSHED + "; %.3f GB of unique K/V per step vs 126 MB L2"
+                        % (work["kv_unique"] / 1e9))
                        if args.flush_l2 else
                        ("inputs larger than L2: %.2f GB of unique K/V per step vs 126 MB L2"
                         % (work["kv_unique"] / 1e9) if work["kv_unique"] > L2_BYTES else
@@ -665,9 +705,7 @@ def run_nvpa(args) -> int:
                       peak_source=peak_source(peaks, "hbm_gbs", "burst copy")),
         e2e=dict(value=work["step"] * world / (e2e_ms * 1e-3) / 1e9, unit="GB/s",
                  h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=e2e_ms,
-                 copies="one packed host-to-device copy of the step's inputs on the step's "
-                        "stream; the read-back of out on a copy stream, overlapping the next "
-                        "step's upload; all inside the timed region",
+                 copies=E2E_COPIES,
                  breakdown_median=e2e_breakdown),
         gpu_launches=int(launches),
         clocks=cs,
@@ -698,7 +736,7 @@ def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
                      dtype=torch.uint8, device=dev)
     out = torch.empty_like(t["q"])
 
-    def one_step(ev=None, inp=None):
+    def one_step(ev=None, inp=None, dst=None):
         inp = t if inp is None else inp
         nvpa.store_kvcache(inp["k_new"], inp["v_new"], t["k_cache"], t["v_cache"],
                            inp["slot_mapping"], stream=stream)
@@ -706,8 +744,8 @@ def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
             ev[0].record(stream)
         nvpa.varlen_prefill_attention(inp["q"], t["k_cache"], t["v_cache"], inp["block_tables"],
                                       inp["cu_seqlens_q"], inp["cu_seqlens_k"], step.max_seqlen_q,
-                                      step.max_seqlen_k, step.scale, out=out, workspace=ws,
-                                      stream=stream)
+                                      step.max_seqlen_k, step.scale, out=out if dst is None else dst,
+                                      workspace=ws, stream=stream)
         if ev is not None:
             ev[1].record(stream)
 
@@ -745,8 +783,8 @@ def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
     # ---------------- end to end: host buffers in, host result out ----------------
     packed = PackedInputs({k: t[k] for k in ("q", "k_new", "v_new", "slot_mapping",
                                              "block_tables", "cu_seqlens_q", "cu_seqlens_k")}, dev)
-    e2e_ms, e2e_breakdown, d2h = end_to_end(lambda inp: one_step(inp=inp), packed, out, stream,
-                                            args.steps, args.warmup, dev)
+    e2e_ms, e2e_breakdown, d2h = end_to_end(lambda inp, o: one_step(inp=inp, dst=o), packed, out,
+                                            stream, args.steps, args.warmup, dev)
     e2e_ms = max_over_ranks(e2e_ms, dev)
     h2d = packed.nbytes
 
@@ -766,7 +804,7 @@ def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
                     num_q_heads=step.num_q_heads, num_kv_heads=step.num_kv_heads,
                     head_dim=step.head_dim, block_size=step.block_size,
                     algorithmic_tflop=work["flops"] / 1e12,
-                    l2=("flushed: a 512 MB write before every step, outside its events"
+                    l2=(L2_FLUSHED
                         if args.flush_l2 else
                         "inputs larger than L2, not flushed: each step stores 101 MB of new K/V "
                         "rows, then reads 101 MB of q and 128 MB of unique K/V and writes 101 MB "
@@ -779,9 +817,7 @@ def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
                       peak_source=peak_source(peaks, "bf16_tflops", "cuBLAS bf16 GEMM, burst")),
         e2e=dict(value=work["flops"] * world / (e2e_ms * 1e-3) / 1e12, unit="TFLOP/s",
                  h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=e2e_ms,
-                 copies="one packed host-to-device copy of the step's inputs on the step's "
-                        "stream; the read-back of out on a copy stream, overlapping the next "
-                        "step's upload; all inside the timed region",
+                 copies=E2E_COPIES,
                  breakdown_median=e2e_breakdown),
         gpu_launches=int(launches), clocks=clocks.summary())
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -805,7 +841,8 @@ def main(argv=None) -> int:
                     help="shared: nvpa_decode_step_shared_prefix; plain: nvpa_decode_step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--flush-l2", action="store_true",
-                    help="write a 512 MB buffer before every timed step (outside its events)")
+                    help="write and read back a 512 MB buffer before every timed step "
+                         "(outside its events)")
     argv = sys.argv[1:] if argv is None else list(argv)
     args = ap.parse_args(argv)
     if args.warmup < 3:

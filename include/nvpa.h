@@ -157,7 +157,7 @@ size_t nvpa_paged_decode_workspace_size(int batch, int num_q_heads, int num_kv_h
  *                   max_context_len (counting full-length contexts) against the 1776
  *                   resident worker warps of a 148-SM B200: small batches get at least
  *                   one item per warp (partitions of 64 keys or more), many sequences
- *                   256-key partitions, a few long sequences about two rounds of items
+ *                   352-key partitions, a few long sequences about two rounds of items
  *                   (128 to 1024 keys); n > 0 = cut the longest possible context into
  *                   at most n partitions (rounded to the library's tile size).
  *   workspace       device scratch of at least nvpa_paged_decode_workspace_size(...)
@@ -279,8 +279,9 @@ nvpa_status_t nvpa_decode_step_shared_prefix(
  *    device again after resetting it in the same process.
  *  - A call whose scratch need (nvpa_paged_decode_workspace_size with the same
  *    arguments) exceeds 64 MiB returns NVPA_ERR_WORKSPACE_TOO_SMALL with a message;
- *    lowering num_splits lowers the need (batch 512 at max_context_len 4096 with 16 query
- *    heads of dim 128 fits with num_splits <= 15).
+ *    lowering num_splits lowers the need (batch 1024 at max_context_len 4096 with 16
+ *    query heads of dim 128 needs 97 MiB with automatic partitioning and fits with
+ *    num_splits <= 7).
  *  - All calls share the one array, which keeps the last call's contents.  Nothing in it
  *    has to start at zero.  Calls whose kernels can overlap on the GPU (different streams
  *    or threads) race on the array: serialise them.

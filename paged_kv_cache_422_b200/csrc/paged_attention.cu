@@ -417,8 +417,12 @@ SharedGeometry shared_geometry(int batch, int hq, int hkv, int max_context_len, 
 // Automatic sizing counts a batch of full-length contexts against kTargetItems, the
 // resident worker warps of a 148-SM B200 (3 CTAs of 4 warps per SM):
 //  - small batches get partitions of 64 keys or more, enough for one item per warp;
-//  - many sequences (more than kTargetItems / 8 sequence-head pairs) keep 256-key
-//    partitions: their lengths vary, and the rounds of items even out by themselves;
+//  - many sequences (more than kTargetItems / 8 sequence-head pairs) get 352-key
+//    partitions: many rounds of items, whose varying lengths even the rounds out; longer
+//    partitions write and merge fewer partials but lengthen the last round (measured on
+//    512 contexts of up to 4 k keys: 352 keys 1 % faster than 256, 688 keys 3 % slower; on
+//    64 contexts of 0.5 to 4 k keys: 336 to 368 keys 3 to 5 % faster than 256, although
+//    288 and 320 keys were 6 and 2 % slower and 504 keys 15 % slower);
 //  - a few long sequences get about two rounds of items, 128 to 1024 keys each: fewer,
 //    longer partitions mean fewer partials to write and merge, and two rounds keep the
 //    warps that idle in the last one a small share (measured on 8 contexts of 32 k keys:
@@ -431,13 +435,14 @@ int decode_chunk_keys(int batch, int num_kv_heads, int max_context_len, int num_
         return std::max(kTileKeys, (per + kTileKeys - 1) / kTileKeys * kTileKeys);
     }
     constexpr long long kTargetItems = 148LL * 3 * kAttnWarps;
-    constexpr long long kMinChunkKeys = 64, kMaxChunkKeys = 256, kMinLongChunk = 128, kMaxLongChunk = 1024;
+    constexpr long long kMinChunkKeys = 64, kFillChunkKeys = 256, kManyChunkKeys = 352;
+    constexpr long long kMinLongChunk = 128, kMaxLongChunk = 1024;
     auto round16 = [](long long k) { return (k + kTileKeys - 1) / kTileKeys * kTileKeys; };
     const long long per_partition = (long long)std::max(1, batch) * std::max(1, num_kv_heads);
     const long long fill = round16((ctx + (kTargetItems + per_partition - 1) / per_partition - 1) /
                                    ((kTargetItems + per_partition - 1) / per_partition));
-    if (fill < kMaxChunkKeys) return (int)std::max(kMinChunkKeys, fill);
-    if (per_partition * 8 > kTargetItems) return (int)kMaxChunkKeys;
+    if (fill < kFillChunkKeys) return (int)std::max(kMinChunkKeys, fill);
+    if (per_partition * 8 > kTargetItems) return (int)kManyChunkKeys;
     const long long parts = (2 * kTargetItems + per_partition - 1) / per_partition;
     const long long chunk = round16((ctx + parts - 1) / parts);
     return (int)std::min(kMaxLongChunk, std::max(kMinLongChunk, chunk));

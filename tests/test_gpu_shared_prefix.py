@@ -34,13 +34,19 @@ def _share(step, donor, members, nblocks):
 
 
 def _prefix_chunk(batch, hkv, max_ctx):
-    """Prefix keys per partition of the shared-prefix step with automatic partitioning:
-    the decode partition (the header's rule: 64 to 256 keys, sized so that a batch of
-    full-length contexts gives about 148 * 3 * 4 work items), rounded up to 128."""
-    per = batch * hkv
-    parts = -(-(148 * 3 * 4) // per)
-    chunk = -(-max_ctx // parts)
-    chunk = min(256, max(64, -(-chunk // 16) * 16))
+    """Prefix keys per partition of the shared-prefix step with automatic partitioning: the
+    decode partition (the header's rule for num_splits = 0), rounded up to 128."""
+    target = 148 * 3 * 4                      # resident worker warps of a 148-SM B200
+    per = max(1, batch) * max(1, hkv)
+    ctx = max(1, max_ctx)
+    r16 = lambda k: -(-k // 16) * 16          # noqa: E731
+    fill = r16(-(-ctx // -(-target // per)))  # one item per warp
+    if fill < 256:
+        chunk = max(64, fill)
+    elif per * 8 > target:
+        chunk = 352
+    else:                                     # about two rounds of items
+        chunk = min(1024, max(128, r16(-(-ctx // -(-2 * target // per)))))
     return -(-chunk // 128) * 128
 
 

@@ -85,10 +85,11 @@ def test_static_scratch_matches_workspace_entry_twice(cuda_device):
 
 def test_static_scratch_rejects_oversized_problem():
     lib = _lib.lib()
-    # batch 512 at 4096 keys with the default partitioning needs more than 64 MiB;
+    # batch 1024 at 4096 keys with the default partitioning needs 97 MiB of the 64;
     # the size check happens before any device work, so null pointers are fine here
+    assert nvpa.paged_decode_workspace_size(1024, 16, 8, 128, 4096, 256, 0) > 64 << 20
     st = lib.nvpa_paged_decode_attention_static_scratch(
-        None, None, None, None, None, None, 16, None, 512, 16, 8, 128, 16384, 256, 4096, 0.1, 0,
+        None, None, None, None, None, None, 16, None, 1024, 16, 8, 128, 16384, 256, 4096, 0.1, 0,
         None, None)
     assert st == _lib.NVPA_ERR_WORKSPACE_TOO_SMALL
     assert b"static scratch holds" in lib.nvpa_last_error()
