@@ -234,7 +234,8 @@ size_t nvpa_decode_shared_prefix_workspace_size(int batch, int num_q_heads, int 
  *  - the worker reads only each member's remaining keys; the combine merges the
  *    prefix and private partitions with their log-sum-exp weights.
  * Sequences in no group are decoded exactly as by nvpa_decode_step.  A batch above
- * 2048 sequences is decoded without groups.  The fused store writes only position
+ * 2048 sequences, or below min_group_size (no group can form), is decoded without
+ * groups, as by nvpa_decode_step.  The fused store writes only position
  * context_lens[b] - 1, which is never inside a group's prefix.
  *
  *   k_new, v_new,   as for nvpa_decode_step, or all three NULL (no store).

@@ -385,7 +385,8 @@ DecodeWorkspace decode_workspace_layout(int batch, int hq, int hkv, int head_dim
 }
 
 // Partitioning of a shared-prefix decode; active == false when the batch is too large
-// for the plan's table (the call then runs as a plain decode step).
+// for the plan's table or smaller than the smallest group (the call then runs as a plain
+// decode step).
 struct SharedGeometry {
     bool active;
     int chunk, s_max, pchunk, ptq, min_members;
@@ -397,13 +398,14 @@ SharedGeometry shared_geometry(int batch, int hq, int hkv, int max_context_len, 
     SharedGeometry g{};
     g.chunk = decode_chunk_keys(batch, hkv, max_context_len, num_splits);
     const int ctx = std::max(0, max_context_len);
-    g.active = batch <= kSharedMaxBatch;
+    g.min_members = min_group > 0 ? std::max(2, min_group) : kDefaultMinGroup;
+    // a batch smaller than the smallest group cannot form one: no plan table, no prefix launch
+    g.active = batch <= kSharedMaxBatch && batch >= g.min_members;
     // one more partition than a plain decode: splitting a context at the prefix boundary
     // adds at most one (pchunk >= chunk)
     g.s_max = std::max(1, (ctx + g.chunk - 1) / g.chunk) + (g.active ? 1 : 0);
     g.pchunk = (g.chunk + 127) / 128 * 128;
     g.ptq = 128 / attention_tile_pack(hq, hkv);
-    g.min_members = min_group > 0 ? std::max(2, min_group) : kDefaultMinGroup;
     const long long groups = batch / g.min_members;
     g.entries = g.active ? ((long long)batch / g.ptq + groups + 1) * ((ctx + g.pchunk - 1) / g.pchunk + 1) : 0;
     return g;

@@ -110,9 +110,10 @@ def test_batch512_shared_prefix_workload(cuda_device):
     (groups, members, tiles), _, _ = _run(step, cuda_device)
     assert groups == 1
     assert members == int(shared.sum())
-    # 1024 prefix keys in 4 partitions of 256; 64 members per query tile (2 query heads
+    # 1024 prefix keys in partitions of pchunk; 64 members per query tile (2 query heads
     # each), query tiles in pairs
-    assert tiles == 4 * (((members + 63) // 64 + 1) // 2)
+    pchunk = _prefix_chunk(step.batch, step.num_kv_heads, step.max_context_len)
+    assert tiles == -(-1024 // pchunk) * (((members + 63) // 64 + 1) // 2)
 
 
 @pytest.mark.parametrize("name", ["decode_tiny_b4", "decode_mid_b64", "decode_long_b8_ctx32k_bs16"])
@@ -133,7 +134,7 @@ def test_shared_prefix_api_on_the_other_decode_workloads(cuda_device, name):
     ([513 + 37 * i for i in range(80)], 16, 8, 128, 256, 70, 2),
     # group of 3 query heads (not a power of two: one head per tile row)
     ([100 + 3 * i for i in range(24)], 6, 2, 128, 32, 20, 3),
-    # group 8: 16 members per tile; 320 prefix keys = 256 + 64
+    # group 8: 16 members per tile; 320 prefix keys (partitions of 128, the last one 64)
     ([330 + 11 * i for i in range(40)], 32, 4, 128, 16, 40, 20),
 ])
 def test_shared_prefix_shapes(cuda_device, lens, hq, hkv, d, bs, nshared, nblk, store):
@@ -182,6 +183,22 @@ def test_small_buckets_are_not_groups(cuda_device):
     share = np.array([True] * 5 + [False] * 7)
     step = make_decode_step(51, lens, num_q_heads=4, num_kv_heads=2, head_dim=64, block_size=16,
                             shared_prefix_blocks=2, share=share)
+    (groups, members, tiles), _, _ = _run(step, cuda_device, min_group=6)
+    assert (groups, members, tiles) == (0, 0, 0)
+    (groups, members, _), _, _ = _run(step, cuda_device, min_group=5)
+    assert (groups, members) == (1, 5)
+
+
+def test_batch_below_the_smallest_group_runs_as_a_plain_step(cuda_device):
+    """A batch of 5 that all share a prefix, with groups of at least 6: no group can form,
+    so the call runs as the plain decode step (no plan table, no prefix launch) and its
+    workspace is the plain step's size."""
+    lens = [90 + 7 * i for i in range(5)]
+    step = make_decode_step(53, lens, num_q_heads=4, num_kv_heads=2, head_dim=64, block_size=16,
+                            shared_prefix_blocks=3, share=np.ones(5, bool))
+    args = (step.batch, step.num_q_heads, step.num_kv_heads, step.head_dim, step.max_context_len,
+            step.block_size, 0)
+    assert nvpa.decode_shared_prefix_workspace_size(*args, 6) == nvpa.paged_decode_workspace_size(*args)
     (groups, members, tiles), _, _ = _run(step, cuda_device, min_group=6)
     assert (groups, members, tiles) == (0, 0, 0)
     (groups, members, _), _, _ = _run(step, cuda_device, min_group=5)
