@@ -669,9 +669,10 @@ def run_nvpa(args) -> int:
     value = work["step"] * world / (ms_step * 1e-3) / 1e9
     attn_gbs = work["step"] / (attn_ms * 1e-3) / 1e9
     traffic = None
-    if args.workload == DEFAULT_WORKLOAD:
-        traffic = profile_traffic("decode_step_shared_prefix_b512" if shared else "decode_worker_b512",
-                                  DECODE_SOURCES)
+    if args.workload == DEFAULT_WORKLOAD and shared:
+        # the worker's DRAM bytes from the committed capture of this step (none is kept for
+        # the plain step's worker)
+        traffic = profile_traffic("decode_step_shared_prefix_b512", DECODE_SOURCES)
     cs = clocks.summary()
     line = dict(
         metric=METRIC, value=value, unit="GB/s", n_gpus=world, steps=args.steps,
