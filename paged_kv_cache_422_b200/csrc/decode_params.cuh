@@ -131,6 +131,8 @@ cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaSt
 cudaError_t launch_decode_plan_shared(const AttnParams& p, cudaStream_t stream);
 // Enqueue the split-KV combine (grid CTAs of 8 warps, one warp per sequence and query
 // head), as a programmatic dependent of the worker.
-cudaError_t launch_decode_combine(const AttnParams& p, int head_dim, int grid, cudaStream_t stream);
+// The split-KV combine over every (sequence, query head) of p (see decode_combine.cu).
+cudaError_t launch_decode_combine(const AttnParams& p, int head_dim, cudaStream_t stream);
+int decode_combine_warps_per_row(long long rows, int s_max);
 
 }  // namespace nvpa

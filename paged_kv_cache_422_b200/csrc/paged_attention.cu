@@ -564,9 +564,7 @@ nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream) {
     e = dispatch_worker(p, c.head_dim, max_items, stream);
     if (e != cudaSuccess) return cuda_failure(e, "decode worker launch");
     if (s_max > 1) {
-        const long long warps = (long long)c.batch * c.hq;
-        const int grid = (int)((warps + 7) / 8);
-        e = launch_decode_combine(p, c.head_dim, grid, stream);
+        e = launch_decode_combine(p, c.head_dim, stream);
         if (e != cudaSuccess) return cuda_failure(e, "decode combine launch");
         count_launches(1);
     }
