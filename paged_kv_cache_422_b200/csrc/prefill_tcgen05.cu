@@ -1,5 +1,6 @@
-// Varlen causal prefill attention on the 5th-generation tensor cores (tcgen05 + TMEM),
-// and the same kernel in the shared-prefix mode of the decode step.
+// Attention on the 5th-generation tensor cores (tcgen05 + TMEM): the varlen causal prefill
+// (prefill_tcgen05_kernel, below) and the shared-prefix tiles of the decode step
+// (prefix_tiles_kernel, further down, where its own description is).
 //
 // ("Nano-vLLM inference engine architecture", section "Low-level performance details":
 // prefill runs a variable-length attention over cumulative sequence lengths; "Nano-vLLM
@@ -110,9 +111,10 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 
 // Columns at or past lim - key0 (keys the row does not see, including rows past the
 // sequence) become -inf by bit mask, whatever they held.
-__device__ __forceinline__ void mask_row(uint32_t (&sv)[kKV], int key0, int lim) {
+template <int N>
+__device__ __forceinline__ void mask_row(uint32_t (&sv)[N], int key0, int lim) {
 #pragma unroll
-    for (int c = 0; c < kKV / 32; ++c) {
+    for (int c = 0; c < N / 32; ++c) {
         const uint32_t vm = visible_mask(lim - key0 - c * 32);
 #pragma unroll
         for (int k = 0; k < 32; ++k) sv[c * 32 + k] = __float_as_uint(keep_or(sv[c * 32 + k], vm, k, -INFINITY));
@@ -121,25 +123,27 @@ __device__ __forceinline__ void mask_row(uint32_t (&sv)[kKV], int key0, int lim)
 
 // Largest value of the row: two independent accumulators, two new values per three-input
 // instruction.
-__device__ __forceinline__ float row_max(const uint32_t (&sv)[kKV]) {
+template <int N>
+__device__ __forceinline__ float row_max(const uint32_t (&sv)[N]) {
     float e0 = -INFINITY, e1 = -INFINITY;
 #pragma unroll
-    for (int k = 0; k < kKV; k += 4) {
+    for (int k = 0; k < N; k += 4) {
         e0 = max3(e0, __uint_as_float(sv[k]), __uint_as_float(sv[k + 1]));
         e1 = max3(e1, __uint_as_float(sv[k + 2]), __uint_as_float(sv[k + 3]));
     }
     return fmaxf(e0, e1);
 }
 
-// P = exp2(s * c + nm) of one row of raw scores (c > 0: the scale in log2 units; one packed
-// FMA per pair of scores), packed to bf16 pairs and written over the first kKV/2 TMEM
-// columns of the row (32 S columns become 16 P columns, each chunk's P landing in columns
-// already read); returns the row sum of the fp32 values.  A -inf score or offset gives 0.
-__device__ __forceinline__ float exp_row(const uint32_t (&sv)[kKV], uint32_t s_col, float c, float nm) {
+// P = exp2(s * c + nm) of N raw scores of a row (c > 0: the scale in log2 units; one
+// packed FMA per pair of scores), packed to bf16 pairs and written to TMEM from column
+// p_col on (32 S columns become 16 P columns); returns the sum of the fp32 values.  A -inf
+// score or offset gives 0.
+template <int N>
+__device__ __forceinline__ float exp_row(const uint32_t (&sv)[N], uint32_t p_col, float c, float nm) {
     const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(nm, nm);
     uint64_t l0 = f2_pack(0.f, 0.f), l1 = l0;
 #pragma unroll
-    for (int cc = 0; cc < kKV / 32; ++cc) {
+    for (int cc = 0; cc < N / 32; ++cc) {
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 32; k += 2) {
@@ -155,7 +159,7 @@ __device__ __forceinline__ float exp_row(const uint32_t (&sv)[kKV], uint32_t s_c
                 l0 = f2_add(l0, p2);
             pk[k / 2] = pack_bf16x2(a, b);
         }
-        tmem_st16(s_col + cc * 16, pk);
+        tmem_st16(p_col + cc * 16, pk);
     }
     float a0, b0, a1, b1;
     f2_unpack(l0, a0, b0);
@@ -401,7 +405,7 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const PrefillParams 
 // ------------------------------------------------------------------------------------
 // the attention kernel
 // ------------------------------------------------------------------------------------
-template <int D, bool PREFIX>
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap k_map,
                        const __grid_constant__ CUtensorMap v_map, const PrefillParams p) {
@@ -417,10 +421,6 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
     UnitDesc* unit_ring = reinterpret_cast<UnitDesc*>(smem + L::RING_OFF);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if constexpr (PREFIX) {
-        // shared-prefix mode: let the decode worker's CTAs launch as this grid's CTAs finish
-        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    }
 
     if (threadIdx.x == 0) {
         for (int x = 0; x < 2; ++x) {
@@ -463,18 +463,11 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
     // overlaps the plan, and nothing the plan writes is read before this wait.
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // Work units: every plan entry for every head group.  In the shared-prefix mode the
-    // work is small (a few groups' prefixes) and latency-bound, so each pair entry is
-    // split into two single-tile units for twice the parallelism.
-    const int total = __ldcg(p.ntiles) * p.hgroups * (PREFIX ? 2 : 1);
+    // Work units: every plan entry (a pair of query tiles) for every head group.
+    const int total = __ldcg(p.ntiles) * p.hgroups;
     auto unit_of = [&](int idx, int4& e, int& hg) {
         hg = idx % p.hgroups;
-        if constexpr (PREFIX) {
-            const int4 pe = __ldg(p.tiles + idx / (2 * p.hgroups));
-            e = make_int4(pe.x, ((idx / p.hgroups) & 1) ? pe.z : pe.y, -1, pe.w);
-        } else {
-            e = __ldg(p.tiles + idx / p.hgroups);
-        }
+        e = __ldg(p.tiles + idx / p.hgroups);
     };
     // Units are claimed dynamically (longest first, as the plan orders them): the producer
     // claims them with an atomic, one unit ahead of the one it loads, and hands each one's
@@ -533,7 +526,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             int4 e;
             int hg;
             entry(resolve(claim_next()), e, hg);
-            cur = describe_unit<PREFIX>(p, e, hg);
+            cur = describe_unit<false>(p, e, hg);
         }
         int pending = claim_next();
         bool ok = true;
@@ -551,11 +544,10 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             int nhg;
             entry(nidx, ne, nhg);
             pending = nidx >= 0 ? claim_next() : total;
-            const TileInfo ta = tile_info<PREFIX>(p, cur, false);
-            const TileInfo tb = tile_info<PREFIX>(p, cur, true);
+            const TileInfo ta = tile_info<false>(p, cur, false);
+            const TileInfo tb = tile_info<false>(p, cur, true);
             const int nkv = max(ta.nkv, tb.nkv);
-            const int bt_seq = PREFIX ? __ldg(p.members + ta.q0) : ta.seq;   // a member's table
-            const int32_t* bt = p.block_tables + (size_t)bt_seq * p.max_blocks;
+            const int32_t* bt = p.block_tables + (size_t)ta.seq * p.max_blocks;
             int cur_blk = load_pieces(bt, ta.kbeg, ta.lk, 0);
             int nxt_blk = nkv > 1 ? load_pieces(bt, ta.kbeg, ta.lk, 1) : kNoPiece;
             // Q tile x of this unit into the next buffer of the Q ring (a buffer frees after
@@ -566,43 +558,11 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                 const uint32_t qs = qfill % kQBufs;
                 if (!mbar_wait(bars + L::B_QEMPTY + qs, ((qfill / kQBufs) & 1) ^ 1, abort_flag, p.err)) return false;
                 uint8_t* qdst = smem + L::Q_OFF + qs * L::TILE_BYTES;
-                if constexpr (PREFIX) {
-                    // gather the members' query rows into the swizzled Q tile with 16-byte
-                    // cp.async copies, all in flight at once: lane l fills rows l, l+32,
-                    // l+64, l+96; row r is member tok0 + r / P, head head0 + r % P, and
-                    // 16-byte chunk c of its 128-byte half goes to chunk c ^ (r % 8) (the
-                    // 128-byte swizzle the MMA descriptors expect).  Rows past the group
-                    // are zero-filled.
-                    const uint16_t* src[kQ / 32];
-#pragma unroll
-                    for (int i = 0; i < kQ / 32; ++i) {
-                        const int r = lane + 32 * i;
-                        const int mi = t.tok0 + (r >> p.pack_shift);
-                        const int b = mi < t.lq ? __ldg(p.members + t.q0 + mi) : -1;
-                        src[i] = b < 0 ? nullptr
-                                       : p.q_rows + ((size_t)b * p.hq + t.head0 + (r & (p.pack - 1))) * D;
-                    }
-#pragma unroll
-                    for (int i = 0; i < kQ / 32; ++i) {
-                        const int r = lane + 32 * i;
-#pragma unroll
-                        for (int c = 0; c < D / 8; ++c) {
-                            uint8_t* dst = qdst + (c / 8) * L::REGION_BYTES + r * 128 + (((c % 8) ^ (r & 7)) * 16);
-                            cp_async16(dst, src[i] != nullptr ? src[i] + c * 8 : p.q_rows, src[i] != nullptr ? 16 : 0);
-                        }
-                    }
-                    cp_async_commit();
-                    cp_async_wait<0>();
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bars + L::B_QFULL + qs);
-                } else {
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(bars + L::B_QFULL + qs, L::TILE_BYTES);
-                        for (int r = 0; r < L::REGIONS; ++r)
-                            tma_load_3d(qdst + r * L::REGION_BYTES, &q_map, bars + L::B_QFULL + qs, r * 64,
-                                        t.head0, t.q0 + t.tok0);
-                    }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bars + L::B_QFULL + qs, L::TILE_BYTES);
+                    for (int r = 0; r < L::REGIONS; ++r)
+                        tma_load_3d(qdst + r * L::REGION_BYTES, &q_map, bars + L::B_QFULL + qs, r * 64,
+                                    t.head0, t.q0 + t.tok0);
                 }
                 ++qfill;
                 return true;
@@ -658,7 +618,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             if (ok && nkv > 0) ok = load_kv(1, 0, cur_blk);
             if (ok) ok = load_q(1);
             // the lengths of the next unit's sequence: these loads overlap this unit's waits
-            const UnitDesc nxt = describe_unit<PREFIX>(p, ne, nhg);
+            const UnitDesc nxt = describe_unit<false>(p, ne, nhg);
             for (int j = 1; j < nkv && ok; ++j) {
                 cur_blk = nxt_blk;
                 nxt_blk = j + 1 < nkv ? load_pieces(bt, ta.kbeg, ta.lk, j + 1) : kNoPiece;
@@ -729,8 +689,8 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
         for (int n = 0; ok; ++n) {
             const UnitDesc u = claim(n);
             if (__shfl_sync(0xffffffffu, u.e.x, 0) < 0) break;
-            const TileInfo ta = tile_info<PREFIX>(p, u, false);
-            const TileInfo tb = tile_info<PREFIX>(p, u, true);
+            const TileInfo ta = tile_info<false>(p, u, false);
+            const TileInfo tb = tile_info<false>(p, u, true);
             // the ring positions follow from these counts: broadcast them (see tmem above)
             const int nk[2] = {__shfl_sync(0xffffffffu, ta.nkv, 0), __shfl_sync(0xffffffffu, tb.nkv, 0)};
             const bool val[2] = {__shfl_sync(0xffffffffu, (int)ta.valid, 0) != 0,
@@ -856,10 +816,10 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
         for (int n = 0;; ++n) {
             const UnitDesc u = claim(n);
             if (u.e.x < 0) break;
-            const TileInfo t = tile_info<PREFIX>(p, u, x == 1);
+            const TileInfo t = tile_info<false>(p, u, x == 1);
             if (t.nkv == 0) continue;
             const int pos = t.lk - t.lq + t.tok0 + rtok;           // absolute position of this row
-            const int lim = (!PREFIX && p.causal) ? min(t.lk, pos + 1) : t.lk;  // keys 0 .. lim-1 visible
+            const int lim = p.causal ? min(t.lk, pos + 1) : t.lk;  // keys 0 .. lim-1 visible
             const int lim_min = __reduce_min_sync(0xffffffffu, lim);
             float m = -INFINITY, l = 0.f;
             bool ok = true;
@@ -880,8 +840,8 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                 tmem_wait_ld();
                 // keys the row does not see at -inf (diagonal tiles only), then the row's
                 // largest value in log2 units (raw scores times a positive factor)
-                if (!open) mask_row(sv, key0, lim);
-                const float mt = row_max(sv) * p.scale_log2;
+                if (!open) mask_row<kKV>(sv, key0, lim);
+                const float mt = row_max<kKV>(sv) * p.scale_log2;
                 const bool over = mt > m + kRescaleSlack;
                 const bool rescale = __any_sync(0xffffffffu, over);
                 float alpha = 1.f;
@@ -894,7 +854,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                 // P_j = exp2(s * scale - m) as bf16 pairs over the first kKV/2 columns of S_j.
                 // A row with no visible key yet (m = -inf) gets exp2(-inf) = 0 through its
                 // offset.
-                l += exp_row(sv, s_col, p.scale_log2, m > -INFINITY ? -m : -INFINITY);
+                l += exp_row<kKV>(sv, s_col, p.scale_log2, m > -INFINITY ? -m : -INFINITY);
                 if (rescale && j > 0) {
                     // O holds P_0..P_{j-1} V (all complete once S_j is): rescale it before
                     // P_j is released to the MMA
@@ -923,16 +883,8 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
             tc_fence_after();
             const bool row_ok = rtok < t.ntok;
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            size_t orow;
-            float* pdst = nullptr;
-            if constexpr (PREFIX) {
-                const int b = row_ok ? __ldg(p.members + t.q0 + t.tok0 + rtok) : 0;
-                orow = ((size_t)b * p.hq + t.head0 + rhead) * p.s_max + t.chunk;
-                pdst = p.o_part + orow * D;
-            } else {
-                orow = (size_t)(t.q0 + t.tok0 + rtok) * p.hq + t.head0 + rhead;
-            }
-            uint4* dst = reinterpret_cast<uint4*>(p.out + (PREFIX ? 0 : orow * D));
+            const size_t orow = (size_t)(t.q0 + t.tok0 + rtok) * p.hq + t.head0 + rhead;
+            uint4* dst = reinterpret_cast<uint4*>(p.out + orow * D);
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
@@ -943,13 +895,7 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                     __syncwarp();
                     if (lane == 0) mbar_arrive(b_ofree);
                 }
-                if (PREFIX && row_ok) {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        __stcg(reinterpret_cast<float4*>(pdst + c * 32 + 4 * q),
-                               make_float4(__uint_as_float(o[4 * q + 0]) * inv, __uint_as_float(o[4 * q + 1]) * inv,
-                                           __uint_as_float(o[4 * q + 2]) * inv, __uint_as_float(o[4 * q + 3]) * inv));
-                } else if (row_ok && p.out_v8) {
+                if (row_ok && p.out_v8) {
                     // 32-byte stores: each fills a whole sector of the output row (a warp's
                     // 32 rows are 32 different lines, so the count of store instructions is
                     // what the epilogue's time goes by)
@@ -974,12 +920,534 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
                     }
                 }
             }
-            if constexpr (PREFIX) {
-                if (row_ok) __stcg(p.lse_part + orow, l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY);
-            } else {
-                if (row_ok && p.lse_out != nullptr) p.lse_out[orow] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
-            }
+            if (row_ok && p.lse_out != nullptr) p.lse_out[orow] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
             pv_before += (uint32_t)t.nkv;
+            ++tcount;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// the shared-prefix tiles of the decode step: one query tile per CTA at a time, two S
+// buffers and Q in TMEM
+// ------------------------------------------------------------------------------------
+// A group of sequences that share a cached prefix ("Nano-vLLM part 1" section 4.2) attends
+// the prefix once: the query rows of a tile are the members' decode queries (128 / P
+// members times the P query heads of one KV head), the keys one partition of the prefix,
+// with no mask but the prefix's length, and each member's result goes to that
+// partition's slot of its split-KV partials for the decode combine.
+//
+// Work unit: ONE query tile.  A group has few tiles and each tile few key tiles, so there
+// is no second tile to overlap with; instead S = Q K_j^T alternates between two TMEM
+// buffers, so S_{j+1} is computed while the softmax still works on S_j: the MMA warp
+// issues O += P_j V_j and S_{j+2} as soon as P_j is ready, and the next softmax finds its
+// S waiting.  Q is kept in TMEM (the A operand of S = Q K^T, like P for O += P V), so the
+// S MMAs read only K from shared memory.  TMEM columns: S buffers [0, 128) and
+// [128, 256), O [256, 256 + D), Q [384, 384 + D / 2) (bf16 pairs).  The two query tiles
+// of a plan entry are consecutive units (claimed by different CTAs at about the same
+// time, so their K/V tiles are read from DRAM once).  Warp roles:
+//   warp 0      TMA producer: K_0, K_1, V_0, K_2, V_1, ... (the order the MMAs read them)
+//               into a 6-stage K/V ring;
+//   warp 1      MMA issuer: S_0, S_1, then O += P_j V_j, S_{j+2} for each key tile j;
+//   warps 2, 3  idle (warpgroup 0's register share goes to the softmax);
+//   warps 4..11 softmax, two warps per row: warps 4..7 keys 0..63 of each key tile and O
+//               columns [0, D/2), warps 8..11 keys 64..127 and O columns [D/2, D); the two
+//               warps of a row exchange its largest score and, at the end, its sum through
+//               shared memory; each warp also stores its half of the row's Q into TMEM.
+constexpr int kStages2 = 6;
+constexpr uint32_t kS2Cols = 128, kO2Col = 256, kQ2Col = 384;
+
+template <int D>
+struct PrefixLayout {
+    static constexpr int REGIONS = D / 64;
+    static constexpr int REGION_BYTES = 128 * 128;
+    static constexpr int TILE_BYTES = REGIONS * REGION_BYTES;
+    static constexpr int STAGE_OFF = 0;
+    static constexpr int BAR_OFF = kStages2 * TILE_BYTES;
+    static constexpr int B_KVFULL = 0, B_KVEMPTY = kStages2, B_SFULL = 2 * kStages2, B_PFULL = B_SFULL + 2;
+    static constexpr int B_ODONE = B_PFULL + 2, B_OFINAL = B_ODONE + 1, B_OFREE = B_OFINAL + 1;
+    static constexpr int B_QREADY = B_OFREE + 1, B_DRAIN = B_QREADY + 1, B_XCH = B_DRAIN + 1;
+    static constexpr int B_UFULL = B_XCH + 4, B_UEMPTY = B_UFULL + kUnitRing;
+    static constexpr int NBARS = B_UEMPTY + kUnitRing;
+    static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+    static constexpr int RING_OFF = (MISC_OFF + 16 + 15) / 16 * 16;
+    static constexpr int XCH_OFF = RING_OFF + 32 * kUnitRing;   // [2 slots][2 halves][128 rows] floats
+    static constexpr int BYTES = XCH_OFF + 2 * 2 * kQ * 4;
+    static constexpr int ALLOC = BYTES + 1024;
+};
+static_assert(PrefixLayout<128>::ALLOC <= 227 * 1024, "shared memory per CTA");
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+prefix_tiles_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap k_map,
+                  const __grid_constant__ CUtensorMap v_map, const PrefillParams p) {
+    using L = PrefixLayout<D>;
+    (void)q_map;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
+    const uint32_t sbase = smem_u32(smem);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+    UnitDesc* unit_ring = reinterpret_cast<UnitDesc*>(smem + L::RING_OFF);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // let the decode worker's CTAs launch as this grid's CTAs finish
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bars + L::B_SFULL + b, 1);
+            mbar_init(bars + L::B_PFULL + b, 8);
+        }
+        mbar_init(bars + L::B_ODONE, 1);
+        mbar_init(bars + L::B_OFINAL, 1);
+        mbar_init(bars + L::B_OFREE, 8);
+        mbar_init(bars + L::B_QREADY, 8);
+        mbar_init(bars + L::B_DRAIN, 1);
+        for (int q = 0; q < 4; ++q) mbar_init(bars + L::B_XCH + q, 2);
+        for (int s = 0; s < kStages2; ++s) {
+            mbar_init(bars + L::B_KVFULL + s, 1);
+            mbar_init(bars + L::B_KVEMPTY + s, 1);
+        }
+        for (int i = 0; i < kUnitRing; ++i) {
+            mbar_init(bars + L::B_UFULL + i, 1);
+            mbar_init(bars + L::B_UEMPTY + i, kUnitReaders);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&k_map);
+        tma_prefetch_desc(&v_map);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
+    // launched as a programmatic dependent of the decode plan: nothing the plan writes is
+    // read before this wait
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    // one unit per query tile: the two tiles of a plan entry, for every head group
+    const int total = __ldcg(p.ntiles) * p.hgroups * 2;
+    auto unit_of = [&](int idx, int4& e, int& hg) {
+        hg = idx % p.hgroups;
+        const int4 pe = __ldg(p.tiles + idx / (2 * p.hgroups));
+        e = make_int4(pe.x, ((idx / p.hgroups) & 1) ? pe.z : pe.y, -1, pe.w);
+    };
+    auto claim = [&](int n) -> UnitDesc {
+        const int slot = n % kUnitRing;
+        UnitDesc u;
+        if (!mbar_wait(bars + L::B_UFULL + slot, (n / kUnitRing) & 1, abort_flag, p.err)) {
+            u.e = make_int4(-2, -1, -1, 0);
+            u.hg = u.q0 = u.lq = u.lk = 0;
+            return u;
+        }
+        u = unit_ring[slot];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + L::B_UEMPTY + slot);
+        return u;
+    };
+
+    if (warp < 4) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kSmallRegs));
+      if (warp == 0) {
+        // ============================ TMA producer ============================
+        uint32_t fill = 0;
+        const int piece = min(p.block_size, kKV);
+        constexpr int kNoPiece = INT_MIN;
+        auto load_pieces = [&](const int32_t* bt, int kbeg, int lk, int j) {
+            const int key0 = j * kKV;
+            const int npieces = (min(kKV, lk - key0) + piece - 1) / piece;
+            return lane < npieces ? __ldg(bt + ((kbeg + key0 + lane * piece) >> p.block_shift)) : kNoPiece;
+        };
+        auto claim_next = [&]() -> int { return lane == 0 ? atomicAdd(p.unit_counter, 1) : 0; };
+        auto resolve = [&](int pending) -> int {
+            const int i = __shfl_sync(0xffffffffu, pending, 0);
+            return i < total ? i : -1;
+        };
+        auto entry = [&](int idx, int4& e, int& hg) {
+            e = make_int4(-1, -1, -1, 0);
+            hg = 0;
+            if (idx >= 0) unit_of(idx, e, hg);
+        };
+        UnitDesc cur;
+        {
+            int4 e;
+            int hg;
+            entry(resolve(claim_next()), e, hg);
+            cur = describe_unit<true>(p, e, hg);
+        }
+        int pending = claim_next();
+        bool ok = true;
+        for (int n = 0; ok; ++n) {
+            const int slot = n % kUnitRing;
+            if (!mbar_wait(bars + L::B_UEMPTY + slot, ((n / kUnitRing) & 1) ^ 1, abort_flag, p.err)) break;
+            if (lane == 0) {
+                unit_ring[slot] = cur;
+                mbar_arrive(bars + L::B_UFULL + slot);
+            }
+            if (cur.e.x < 0) break;
+            const int nidx = resolve(pending);
+            int4 ne;
+            int nhg;
+            entry(nidx, ne, nhg);
+            pending = nidx >= 0 ? claim_next() : total;
+            const TileInfo ta = tile_info<true>(p, cur, false);
+            const int nkv = ta.nkv;
+            // the prefix's blocks are the same in every member's table: read the first member's
+            const int32_t* bt = p.block_tables + (size_t)__ldg(p.members + ta.q0) * p.max_blocks;
+            // K (kv = 0) or V tile j into the next ring stage; lane c holds piece c's block id
+            auto load_kv = [&](int kv, int j, int blk_lane) -> bool {
+                const int slot = fill % kStages2;
+                if (!mbar_wait(bars + L::B_KVEMPTY + slot, ((fill / kStages2) & 1) ^ 1, abort_flag, p.err))
+                    return false;
+                const bool in_range = blk_lane >= 0 && blk_lane < p.num_blocks;
+                if (kv == 0 && blk_lane != kNoPiece && !in_range) flag_error(p.err, NVPA_FLAG_BAD_BLOCK_ID);
+                const uint32_t valid_mask = __ballot_sync(0xffffffffu, in_range);
+                const uint32_t bytes = (uint32_t)__popc(valid_mask) * (uint32_t)(piece * 128 * L::REGIONS);
+                uint8_t* dst = smem + L::STAGE_OFF + slot * L::TILE_BYTES;
+                const uint32_t bad_mask = __ballot_sync(0xffffffffu, blk_lane != kNoPiece && !in_range);
+                if (bad_mask != 0) {
+                    for (uint32_t m = bad_mask; m != 0; m &= m - 1) {
+                        const int c = __ffs(m) - 1;
+                        for (int r = 0; r < L::REGIONS; ++r) {
+                            uint4* rows = reinterpret_cast<uint4*>(dst + r * L::REGION_BYTES + c * piece * 128);
+                            for (int k = lane; k < piece * 8; k += 32) rows[k] = make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                const CUtensorMap* map = kv ? &v_map : &k_map;
+                if (lane == 0) mbar_arrive_expect_tx(bars + L::B_KVFULL + slot, bytes);
+                for (uint32_t m = valid_mask; m != 0; m &= m - 1) {
+                    const int c = __ffs(m) - 1;
+                    const int blk = __shfl_sync(0xffffffffu, blk_lane, c);
+                    if (lane == 0) {
+                        const int kc = ta.kbeg + j * kKV + c * piece;
+                        const int z = blk * p.block_size + (kc & (p.block_size - 1));
+                        for (int r = 0; r < L::REGIONS; ++r)
+                            tma_load_3d(dst + r * L::REGION_BYTES + c * piece * 128, map, bars + L::B_KVFULL + slot,
+                                        r * 64, ta.hk, z);
+                    }
+                }
+                ++fill;
+                return true;
+            };
+            if (nkv > 0) {
+                int blk0 = load_pieces(bt, ta.kbeg, ta.lk, 0);
+                int blk1 = nkv > 1 ? load_pieces(bt, ta.kbeg, ta.lk, 1) : kNoPiece;
+                ok = load_kv(0, 0, blk0);
+                for (int j = 0; j < nkv && ok; ++j) {
+                    const int blk2 = j + 2 < nkv ? load_pieces(bt, ta.kbeg, ta.lk, j + 2) : kNoPiece;
+                    if (j + 1 < nkv) ok = load_kv(0, j + 1, blk1);
+                    if (ok) ok = load_kv(1, j, blk0);
+                    blk0 = blk1;
+                    blk1 = blk2;
+                }
+            }
+            cur = describe_unit<true>(p, ne, nhg);
+        }
+        if (lane == 0) {
+            for (uint32_t s = 0; s < (uint32_t)kStages2; ++s) {
+                if (fill <= s) continue;
+                const uint32_t last = fill - 1 - (fill - 1 - s) % kStages2;
+                const uint64_t t0 = global_ns();
+                while (!mbar_try_wait(bars + L::B_KVFULL + s, (last / kStages2) & 1) &&
+                       global_ns() - t0 < 100000000ull) {
+                }
+            }
+        }
+      } else if (warp == 1) {
+        // ============================ MMA issuer ============================
+        const uint32_t IDESC_S = idesc_bf16_f32(kQ, kKV, false) | (p.negate_qk ? (1u << 13) : 0u);
+        constexpr uint32_t IDESC_PV = idesc_bf16_f32(kQ, D, true);
+        constexpr uint32_t DESC_HI = sdesc_sw128_hi(1024);
+        constexpr uint32_t TILE16 = L::TILE_BYTES >> 4, REGION16 = L::REGION_BYTES >> 4;
+        const uint32_t k_lo = sdesc_sw128_lo(sbase + L::STAGE_OFF, 16);
+        const uint32_t v_lo = sdesc_sw128_lo(sbase + L::STAGE_OFF, L::REGION_BYTES);
+        uint32_t fill = 0;     // ring entries consumed, in the producer's order
+        uint32_t g = 0;        // key tiles so far (S buffer of key tile j: (g + j) & 1)
+        uint32_t qcount = 0;   // units with work
+        bool ok = true;
+        auto take = [&](uint32_t& slot) -> bool {
+            slot = fill % kStages2;
+            const bool r = mbar_wait(bars + L::B_KVFULL + slot, (fill / kStages2) & 1, abort_flag, p.err);
+            ++fill;
+            return r;
+        };
+        auto issue_s = [&](uint32_t buf, uint32_t kslot) {
+            const uint32_t b = k_lo + kslot * TILE16;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t o = (kk / 4) * REGION16 + (kk % 4) * 2;
+                umma_ts(tmem + buf * kS2Cols, tmem + kQ2Col + kk * 8, sdesc_join(b + o, DESC_HI), IDESC_S,
+                        kk > 0 ? 1u : 0u);
+            }
+            umma_commit(bars + L::B_SFULL + buf);
+            umma_commit(bars + L::B_KVEMPTY + kslot);
+        };
+        auto issue_pv = [&](uint32_t buf, uint32_t vslot, bool accumulate) {
+            const uint32_t b = v_lo + vslot * TILE16;
+#pragma unroll
+            for (int kk = 0; kk < kKV / 16; ++kk)
+                umma_ts(tmem + kO2Col, tmem + buf * kS2Cols + kk * 8, sdesc_join(b + kk * 128, DESC_HI), IDESC_PV,
+                        (accumulate || kk > 0) ? 1u : 0u);
+            umma_commit(bars + L::B_ODONE);
+            umma_commit(bars + L::B_KVEMPTY + vslot);
+        };
+        for (int n = 0; ok; ++n) {
+            const UnitDesc u = claim(n);
+            if (__shfl_sync(0xffffffffu, u.e.x, 0) < 0) break;
+            const TileInfo t = tile_info<true>(p, u, false);
+            const int nk = __shfl_sync(0xffffffffu, t.nkv, 0);
+            const int lk = __shfl_sync(0xffffffffu, t.lk, 0);
+            if (nk == 0) continue;
+            // this unit's Q is in TMEM
+            if (!mbar_wait(bars + L::B_QREADY, qcount & 1, abort_flag, p.err)) break;
+            uint32_t slot;
+            if (!take(slot)) break;
+            tc_fence_after();
+            if (lane == 0) issue_s(g & 1, slot);
+            __syncwarp();
+            if (nk > 1) {
+                if (!take(slot)) break;
+                tc_fence_after();
+                if (lane == 0) issue_s((g + 1) & 1, slot);
+                __syncwarp();
+            }
+            for (int j = 0; j < nk && ok; ++j) {
+                const uint32_t b = (g + j) & 1;
+                if (!mbar_wait(bars + L::B_PFULL + b, ((g + j) >> 1) & 1, abort_flag, p.err)) {
+                    ok = false;
+                    break;
+                }
+                if (j == 0 && qcount > 0 && !mbar_wait(bars + L::B_OFREE, (qcount - 1) & 1, abort_flag, p.err)) {
+                    ok = false;
+                    break;
+                }
+                uint32_t vslot;
+                if (!take(vslot)) {
+                    ok = false;
+                    break;
+                }
+                const int valid = min(kKV, lk - j * kKV);
+                if (valid < kKV) {
+                    // zero the V rows past the sequence (stale cache rows, or never loaded)
+                    uint8_t* vt = smem + L::STAGE_OFF + vslot * L::TILE_BYTES;
+                    for (int r = 0; r < L::REGIONS; ++r) {
+                        uint4* rowp = reinterpret_cast<uint4*>(vt + r * L::REGION_BYTES + valid * 128);
+                        const int n16 = (kKV - valid) * 8;
+                        for (int k = lane; k < n16; k += 32) rowp[k] = make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    issue_pv(b, vslot, j > 0);
+                    if (j == nk - 1) umma_commit(bars + L::B_OFINAL);
+                }
+                __syncwarp();
+                if (j + 2 < nk) {
+                    // S_{j+2} into the buffer whose P_j the P V just issued reads first
+                    uint32_t kslot;
+                    if (!take(kslot)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (lane == 0) issue_s(b, kslot);
+                    __syncwarp();
+                }
+            }
+            g += (uint32_t)nk;
+            ++qcount;
+        }
+        if (lane == 0) umma_commit(bars + L::B_DRAIN);
+        __syncwarp();
+        const uint64_t t0 = global_ns();
+        while (!mbar_try_wait(bars + L::B_DRAIN, 0) && global_ns() - t0 < 100000000ull) {
+        }
+      }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+        // ============================ softmax warps ============================
+        constexpr int NC = kKV / 2;                    // S columns of this warp
+        constexpr int DC = D / 2;                      // O columns of this warp
+        const int h = (warp - 4) >> 2;                 // column half
+        const int quarter = warp & 3;                  // TMEM lanes 32*quarter .. +31
+        const int r = quarter * 32 + lane;
+        const int rtok = r >> p.pack_shift;
+        const int rhead = r & (p.pack - 1);
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        const uint32_t s_base = tmem + lane_base;
+        const uint32_t o_col = tmem + lane_base + kO2Col + h * DC;
+        const uint32_t q_col = tmem + lane_base + kQ2Col + h * (D / 4);
+        float* xch = reinterpret_cast<float*>(smem + L::XCH_OFF);
+        uint64_t* b_xch = bars + L::B_XCH + quarter;
+        uint32_t x_use = 0;
+        // Publish v, wait for the partner warp of the row, return its value.  Two slots by
+        // use parity: a warp can be one exchange ahead of its partner's read, never two.
+        auto exchange = [&](float v, float& other) -> bool {
+            const int sl = (int)(x_use & 1);
+            xch[(sl * 2 + h) * kQ + r] = v;
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b_xch);
+            if (!mbar_wait(b_xch, x_use & 1, abort_flag, p.err)) return false;
+            ++x_use;
+            tc_fence_after();
+            other = xch[(sl * 2 + (h ^ 1)) * kQ + r];
+            return true;
+        };
+        uint32_t g = 0;
+        int tcount = 0;
+        uint32_t pv_before = 0;
+        for (int n = 0;; ++n) {
+            const UnitDesc u = claim(n);
+            if (u.e.x < 0) break;
+            const TileInfo t = tile_info<true>(p, u, false);
+            if (t.nkv == 0) continue;
+            const bool row_ok = rtok < t.ntok;
+            // this warp's half of the row's Q into TMEM (zeros for rows past the tile); the
+            // previous unit's S MMAs, which read Q, have all completed (each was waited for)
+            {
+                // row r: member tok0 + r / P of the group, query head head0 + r % P
+                const uint16_t* src = nullptr;
+                if (row_ok) {
+                    const int b = __ldg(p.members + t.q0 + t.tok0 + rtok);
+                    src = p.q_rows + ((size_t)b * p.hq + t.head0 + rhead) * D;
+                }
+                uint32_t qw[D / 4];   // D / 2 bf16: D / 16 loads of 16 bytes
+#pragma unroll
+                for (int c = 0; c < D / 16; ++c) {
+                    const uint4 v = src != nullptr ? __ldg(reinterpret_cast<const uint4*>(src + h * DC) + c)
+                                                   : make_uint4(0, 0, 0, 0);
+                    qw[4 * c + 0] = v.x;
+                    qw[4 * c + 1] = v.y;
+                    qw[4 * c + 2] = v.z;
+                    qw[4 * c + 3] = v.w;
+                }
+                if constexpr (D / 4 == 32) {
+                    tmem_st32(q_col, qw);
+                } else {
+                    tmem_st16(q_col, qw);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars + L::B_QREADY);
+            }
+            // every member sees all of the prefix: only keys past its length are masked
+            const int lim = t.lk;
+            const int lim_min = lim;
+            float m = -INFINITY, l = 0.f;
+            bool ok = true;
+            for (int j = 0; j < t.nkv; ++j) {
+                const uint32_t b = (g + j) & 1;
+                if (!mbar_wait(bars + L::B_SFULL + b, ((g + j) >> 1) & 1, abort_flag, p.err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int key0 = j * kKV;
+                const bool open = key0 + kKV <= lim_min;
+                const uint32_t s_col = s_base + b * kS2Cols;
+                uint32_t sv[NC];
+#pragma unroll
+                for (int c = 0; c < NC / 32; ++c)
+                    tmem_ld32(s_col + h * NC + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
+                tmem_wait_ld();
+                if (!open) mask_row<NC>(sv, key0 + h * NC, lim);
+                float mt = row_max<NC>(sv) * p.scale_log2;
+                {
+                    float mo;
+                    if (!exchange(mt, mo)) {
+                        ok = false;
+                        break;
+                    }
+                    mt = fmaxf(mt, mo);
+                }
+                const bool over = mt > m + kRescaleSlack;
+                const bool rescale = __any_sync(0xffffffffu, over);
+                float alpha = 1.f;
+                if (rescale) {
+                    const float m_new = over ? mt : m;
+                    alpha = over ? (m == -INFINITY ? 0.f : fast_exp2(m - m_new)) : 1.f;
+                    l *= alpha;
+                    m = m_new;
+                }
+                l += exp_row<NC>(sv, s_col + h * (NC / 2), p.scale_log2, m > -INFINITY ? -m : -INFINITY);
+                if (rescale && j > 0) {
+                    // O holds P_0..P_{j-1} V: wait for the last of those, then rescale this
+                    // warp's columns before P_j is released
+                    if (!mbar_wait(bars + L::B_ODONE, (pv_before + j - 1) & 1, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int c = 0; c < DC / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(o_col + c * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                        tmem_st32(o_col + c * 32, o);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars + L::B_PFULL + b);
+            }
+            if (!ok) break;
+            if (!mbar_wait(bars + L::B_OFINAL, tcount & 1, abort_flag, p.err)) break;
+            tc_fence_after();
+            {
+                float lo;
+                if (!exchange(l, lo)) break;
+                l += lo;
+            }
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            // partition `chunk` of the prefix goes to slot `chunk` of each member's partials
+            const int b = row_ok ? __ldg(p.members + t.q0 + t.tok0 + rtok) : 0;
+            const size_t orow = ((size_t)b * p.hq + t.head0 + rhead) * p.s_max + t.chunk;
+            float* pdst = p.o_part + orow * D;
+#pragma unroll
+            for (int c = 0; c < DC / 32; ++c) {
+                const int cg = h * (DC / 32) + c;   // 32-column chunk of the O row
+                uint32_t o[32];
+                tmem_ld32(o_col + c * 32, o);
+                tmem_wait_ld();
+                if (c == DC / 32 - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bars + L::B_OFREE);
+                }
+                if (row_ok) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        __stcg(reinterpret_cast<float4*>(pdst + cg * 32 + 4 * q),
+                               make_float4(__uint_as_float(o[4 * q + 0]) * inv, __uint_as_float(o[4 * q + 1]) * inv,
+                                           __uint_as_float(o[4 * q + 2]) * inv, __uint_as_float(o[4 * q + 3]) * inv));
+                }
+            }
+            if (row_ok && h == 0) __stcg(p.lse_part + orow, l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY);
+            pv_before += (uint32_t)t.nkv;
+            g += (uint32_t)t.nkv;
             ++tcount;
         }
     }
@@ -1037,6 +1505,17 @@ bool make_map(CUtensorMap* map, const void* base, int dim, int heads, long long 
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The varlen prefill runs pairs of query tiles (prefill_tcgen05_kernel); the shared-prefix
+// tiles of the decode step run one query tile at a time with two S buffers
+// (prefix_tiles_kernel).  Both take the same arguments.
+template <int D, bool PREFIX>
+constexpr auto prefill_kernel_fn() {
+    if constexpr (PREFIX) return prefix_tiles_kernel<D>;
+    else return prefill_tcgen05_kernel<D>;
+}
+template <int D, bool PREFIX>
+constexpr int prefill_smem() { return PREFIX ? PrefixLayout<D>::ALLOC : Layout<D>::ALLOC; }
+
 template <int D, bool PREFIX>
 cudaError_t launch_prefill(const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
                            const PrefillParams& p, int grid, cudaStream_t stream, bool pdl = PREFIX) {
@@ -1045,11 +1524,11 @@ cudaError_t launch_prefill(const CUtensorMap& qm, const CUtensorMap& km, const C
     int dev = 0;
     cudaGetDevice(&dev);
     std::call_once(once[dev & 63], [dev] {
-        cudaFuncSetAttribute(prefill_tcgen05_kernel<D, PREFIX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Layout<D>::ALLOC);
+        cudaFuncSetAttribute(prefill_kernel_fn<D, PREFIX>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             prefill_smem<D, PREFIX>());
         cudaFuncAttributes fa{};
         launch_regs[dev & 63] =
-            cudaFuncGetAttributes(&fa, prefill_tcgen05_kernel<D, PREFIX>) == cudaSuccess ? fa.numRegs : 0;
+            cudaFuncGetAttributes(&fa, prefill_kernel_fn<D, PREFIX>()) == cudaSuccess ? fa.numRegs : 0;
     });
     // The warpgroups' setmaxnreg shares add up to kLaunchRegs per thread: with fewer registers
     // at launch the raising warpgroups could never get their share, so do not launch.
@@ -1059,20 +1538,21 @@ cudaError_t launch_prefill(const CUtensorMap& qm, const CUtensorMap& km, const C
         return cudaErrorInvalidConfiguration;
     }
     if (!pdl) {
-        prefill_tcgen05_kernel<D, PREFIX><<<grid, kThreads, Layout<D>::ALLOC, stream>>>(qm, km, vm, p);
+        auto kern = prefill_kernel_fn<D, PREFIX>();
+        kern<<<grid, kThreads, prefill_smem<D, PREFIX>(), stream>>>(qm, km, vm, p);
         return cudaGetLastError();
     } else {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(grid);
         cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = Layout<D>::ALLOC;
+        cfg.dynamicSmemBytes = prefill_smem<D, PREFIX>();
         cfg.stream = stream;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, prefill_tcgen05_kernel<D, PREFIX>, qm, km, vm, p);
+        return cudaLaunchKernelEx(&cfg, prefill_kernel_fn<D, PREFIX>(), qm, km, vm, p);
     }
 }
 
@@ -1157,6 +1637,7 @@ nvpa_status_t run_varlen_prefill_tcgen05(const PrefillCall& c, void* workspace, 
     p.cu_q = c.cu_seqlens_q;
     p.cu_k = c.cu_seqlens_k;
     p.out = static_cast<uint16_t*>(c.out);
+    p.q_rows = static_cast<const uint16_t*>(c.q);   // the query rows, read directly by one kernel form
     p.lse_out = c.lse_out;
     p.err = c.err_flag;
     p.ntiles = reinterpret_cast<int32_t*>(ws);
