@@ -233,7 +233,7 @@ static_assert(Layout<128>::ALLOC <= 227 * 1024, "shared memory per CTA");
 struct UnitDesc {
     int4 e;              // plan entry: sequence (group), query tile A, tile B or -1, key partition
     int hg;              // head group
-    int q0, lq, lk;      // first query row, query rows, keys (prefix mode: prefix length)
+    int q0, lq, lk;      // first query row, query rows, keys (shared-prefix tiles: prefix length)
 };
 static_assert(sizeof(UnitDesc) == 32, "unit description size");
 
@@ -241,7 +241,7 @@ struct TileInfo {
     bool valid;          // false: the pair's B slot is empty
     int seq, qt, head0, hk;
     int q0, lq, lk;      // first query row (global), query rows, keys of the sequence
-    int kbeg, chunk;     // shared-prefix mode: first key and index of the key partition
+    int kbeg, chunk;     // shared-prefix tiles: first key and index of the key partition
     int tok0, ntok;      // first token of the tile inside the sequence, tokens in the tile
     int nkv;             // key tiles visited
 };
