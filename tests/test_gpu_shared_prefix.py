@@ -151,6 +151,22 @@ def test_shared_prefix_shapes(cuda_device, lens, hq, hkv, d, bs, nshared, nblk, 
     assert tiles == -(-nblk * bs // pchunk) * ((-(-nshared // tq) + 1) // 2)   # query-tile pairs
 
 
+def test_prefix_partitions_of_two_key_tiles(cuda_device):
+    """16 contexts up to 4096 keys with 8 KV heads get 160-key decode partitions, so the
+    prefix partitions are 256 keys: every prefix tile unit runs two key tiles, one in each
+    of the kernel's two S buffers, before its epilogue."""
+    lens = [4096 - 37 * i for i in range(16)]
+    share = np.array([i % 4 != 3 for i in range(16)])
+    step = make_decode_step(33, lens, num_q_heads=16, num_kv_heads=8, head_dim=128,
+                            block_size=64, shared_prefix_blocks=8, share=share)
+    pchunk = _prefix_chunk(step.batch, 8, step.max_context_len)
+    assert pchunk == 256
+    (groups, members, tiles), _, _ = _run(step, cuda_device, min_group=4)
+    assert (groups, members) == (1, 12)
+    # 512 prefix keys in two partitions, 12 members in one query tile (a pair of one)
+    assert tiles == 2
+
+
 def test_two_groups_and_a_short_common_run(cuda_device):
     """Two groups with different donors; one member of the second group shares only two
     of the donor's four blocks, so that group's prefix is two blocks."""
