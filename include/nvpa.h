@@ -158,8 +158,9 @@ size_t nvpa_paged_decode_workspace_size(int batch, int num_q_heads, int num_kv_h
  *                   resident worker warps of a 148-SM B200: small batches get at least
  *                   one item per warp (partitions of 64 keys or more), many sequences
  *                   352-key partitions, a few long sequences about two rounds of items
- *                   (128 to 1024 keys); n > 0 = cut the longest possible context into
- *                   at most n partitions (rounded to the library's tile size).
+ *                   (128 to 1024 keys, at most 32 cache blocks); n > 0 = cut the longest
+ *                   possible context into at most n partitions (rounded to the library's
+ *                   tile size).
  *   workspace       device scratch of at least nvpa_paged_decode_workspace_size(...)
  *                   bytes, 256-byte aligned; contents need no initialisation and are
  *                   overwritten.  Calls that share a workspace must not overlap.

@@ -73,7 +73,7 @@ extern "C" nvpa_status_t nvpa_paged_decode_attention_static_scratch(
         return NVPA_ERR_INVALID_ARG;
     }
     const size_t need = decode_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim,
-                                               max_context_len, num_splits);
+                                               max_context_len, block_size, num_splits);
     if (need > kStaticScratchBytes) {
         set_error("static scratch holds %zu bytes but this call needs %zu: lower num_splits or the "
                   "batch, or pass a workspace to nvpa_paged_decode_attention",

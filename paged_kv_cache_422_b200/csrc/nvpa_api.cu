@@ -129,12 +129,11 @@ nvpa_status_t nvpa_store_kvcache(const void* k, const void* v, int64_t k_token_s
 
 size_t nvpa_paged_decode_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim,
                                         int max_context_len, int block_size, int num_splits) {
-    (void)block_size;
     if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_context_len < 0 ||
         num_splits < 0)
         return 0;
     return decode_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_context_len,
-                                  num_splits);
+                                  block_size, num_splits);
 }
 
 nvpa_status_t nvpa_paged_decode_attention(void* out, float* lse_out, const void* q,
@@ -236,12 +235,11 @@ nvpa_status_t nvpa_decode_step(void* out, float* lse_out, const void* q, const v
 size_t nvpa_decode_shared_prefix_workspace_size(int batch, int num_q_heads, int num_kv_heads,
                                                 int head_dim, int max_context_len, int block_size,
                                                 int num_splits, int min_group_size) {
-    (void)block_size;
     if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_context_len < 0 ||
         num_splits < 0 || min_group_size < 0 || num_q_heads % num_kv_heads != 0)
         return 0;
     return decode_shared_prefix_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim,
-                                                max_context_len, num_splits, min_group_size);
+                                                max_context_len, block_size, num_splits, min_group_size);
 }
 
 nvpa_status_t nvpa_decode_step_shared_prefix(

@@ -91,11 +91,12 @@ struct DecodePrefixArgs {
 int attention_tile_pack(int hq, int hkv);
 cudaError_t launch_decode_prefix_tcgen05(const DecodePrefixArgs& a, cudaStream_t stream);
 
-int decode_chunk_keys(int batch, int num_kv_heads, int max_context_len, int num_splits);
+int decode_chunk_keys(int batch, int num_kv_heads, int max_context_len, int block_size, int num_splits);
 size_t decode_workspace_bytes(int batch, int hq, int hkv, int head_dim, int max_context_len,
-                              int num_splits);
+                              int block_size, int num_splits);
 size_t decode_shared_prefix_workspace_bytes(int batch, int hq, int hkv, int head_dim,
-                                            int max_context_len, int num_splits, int min_group);
+                                            int max_context_len, int block_size, int num_splits,
+                                            int min_group);
 nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream);
 size_t prefill_workspace_bytes(int batch, int total_q);
 nvpa_status_t run_varlen_prefill_tcgen05(const PrefillCall& c, void* workspace, size_t workspace_bytes,

@@ -393,10 +393,10 @@ struct SharedGeometry {
     long long entries;   // bound on prefix tile entries
 };
 
-SharedGeometry shared_geometry(int batch, int hq, int hkv, int max_context_len, int num_splits,
-                               int min_group) {
+SharedGeometry shared_geometry(int batch, int hq, int hkv, int max_context_len, int block_size,
+                               int num_splits, int min_group) {
     SharedGeometry g{};
-    g.chunk = decode_chunk_keys(batch, hkv, max_context_len, num_splits);
+    g.chunk = decode_chunk_keys(batch, hkv, max_context_len, block_size, num_splits);
     const int ctx = std::max(0, max_context_len);
     g.min_members = min_group > 0 ? std::max(2, min_group) : kDefaultMinGroup;
     // a batch smaller than the smallest group cannot form one: no plan table, no prefix launch
@@ -425,12 +425,15 @@ SharedGeometry shared_geometry(int batch, int hq, int hkv, int max_context_len, 
 //    512 contexts of up to 4 k keys: 352 keys 1 % faster than 256, 688 keys 3 % slower; on
 //    64 contexts of 0.5 to 4 k keys: 336 to 368 keys 3 to 5 % faster than 256, although
 //    288 and 320 keys were 6 and 2 % slower and 504 keys 15 % slower);
-//  - a few long sequences get about two rounds of items, 128 to 1024 keys each: fewer,
-//    longer partitions mean fewer partials to write and merge, and two rounds keep the
-//    warps that idle in the last one a small share (measured on 8 contexts of 32 k keys:
-//    592-key partitions beat 256-key ones by 6 %, 240-key ones lost 6 %; on 16 contexts of
+//  - a few long sequences get about two rounds of items, 128 to 1024 keys each and at
+//    most 32 cache blocks: fewer, longer partitions mean fewer partials to write and
+//    merge, and two rounds keep the warps that idle in the last one a small share; a
+//    worker warp holds one block id per lane for its partition, so a partition of more
+//    than 32 blocks looks its later blocks up one key tile at a time, on the copy's path
+//    (measured on 8 contexts of 32 k keys in blocks of 16: 512-key partitions 0.205 ms per
+//    step, 592 keys (37 blocks) 0.217, 464 keys 0.213, 256 keys 0.228; on 16 contexts of
 //    4 k keys 160-key partitions beat 256-key ones by 12 %).
-int decode_chunk_keys(int batch, int num_kv_heads, int max_context_len, int num_splits) {
+int decode_chunk_keys(int batch, int num_kv_heads, int max_context_len, int block_size, int num_splits) {
     const int ctx = std::max(1, max_context_len);
     if (num_splits > 0) {
         const int per = (ctx + num_splits - 1) / num_splits;
@@ -447,28 +450,30 @@ int decode_chunk_keys(int batch, int num_kv_heads, int max_context_len, int num_
     if (per_partition * 8 > kTargetItems) return (int)kManyChunkKeys;
     const long long parts = (2 * kTargetItems + per_partition - 1) / per_partition;
     const long long chunk = round16((ctx + parts - 1) / parts);
-    return (int)std::min(kMaxLongChunk, std::max(kMinLongChunk, chunk));
+    const long long cap = std::min(kMaxLongChunk, std::max(kMinLongChunk, 32LL * std::max(1, block_size)));
+    return (int)std::min(cap, std::max(kMinLongChunk, chunk));
 }
 
 size_t decode_workspace_bytes(int batch, int hq, int hkv, int head_dim, int max_context_len,
-                              int num_splits) {
-    const int chunk = decode_chunk_keys(batch, hkv, max_context_len, num_splits);
+                              int block_size, int num_splits) {
+    const int chunk = decode_chunk_keys(batch, hkv, max_context_len, block_size, num_splits);
     const int s_max = std::max(1, (std::max(0, max_context_len) + chunk - 1) / chunk);
     return decode_workspace_layout(batch, hq, hkv, head_dim, s_max).total;
 }
 
 size_t decode_shared_prefix_workspace_bytes(int batch, int hq, int hkv, int head_dim,
-                                            int max_context_len, int num_splits, int min_group) {
-    const SharedGeometry g = shared_geometry(batch, hq, hkv, max_context_len, num_splits, min_group);
+                                            int max_context_len, int block_size, int num_splits,
+                                            int min_group) {
+    const SharedGeometry g = shared_geometry(batch, hq, hkv, max_context_len, block_size, num_splits, min_group);
     return decode_workspace_layout(batch, hq, hkv, head_dim, g.s_max, g.entries).total;
 }
 
 nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream) {
     const SharedGeometry sg = c.shared_prefix
-        ? shared_geometry(c.batch, c.hq, c.hkv, c.max_context_len, c.num_splits, c.min_group)
+        ? shared_geometry(c.batch, c.hq, c.hkv, c.max_context_len, c.block_size, c.num_splits, c.min_group)
         : SharedGeometry{};
     const bool shared = c.shared_prefix && sg.active;
-    const int chunk = decode_chunk_keys(c.batch, c.hkv, c.max_context_len, c.num_splits);
+    const int chunk = decode_chunk_keys(c.batch, c.hkv, c.max_context_len, c.block_size, c.num_splits);
     const int s_max = c.shared_prefix ? sg.s_max : std::max(1, (std::max(0, c.max_context_len) + chunk - 1) / chunk);
     const DecodeWorkspace w = decode_workspace_layout(c.batch, c.hq, c.hkv, c.head_dim, s_max, sg.entries);
     if (c.workspace_bytes < w.total) {

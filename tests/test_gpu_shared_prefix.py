@@ -33,7 +33,7 @@ def _share(step, donor, members, nblocks):
     return step
 
 
-def _prefix_chunk(batch, hkv, max_ctx):
+def _prefix_chunk(batch, hkv, max_ctx, block_size):
     """Prefix keys per partition of the shared-prefix step with automatic partitioning: the
     decode partition (the header's rule for num_splits = 0), rounded up to 128."""
     target = 148 * 3 * 4                      # resident worker warps of a 148-SM B200
@@ -45,8 +45,9 @@ def _prefix_chunk(batch, hkv, max_ctx):
         chunk = max(64, fill)
     elif per * 8 > target:
         chunk = 352
-    else:                                     # about two rounds of items
-        chunk = min(1024, max(128, r16(-(-ctx // -(-2 * target // per)))))
+    else:                                     # about two rounds of items, <= 32 blocks
+        cap = min(1024, max(128, 32 * block_size))
+        chunk = min(cap, max(128, r16(-(-ctx // -(-2 * target // per)))))
     return -(-chunk // 128) * 128
 
 
@@ -112,7 +113,7 @@ def test_batch512_shared_prefix_workload(cuda_device):
     assert members == int(shared.sum())
     # 1024 prefix keys in partitions of pchunk; 64 members per query tile (2 query heads
     # each), query tiles in pairs
-    pchunk = _prefix_chunk(step.batch, step.num_kv_heads, step.max_context_len)
+    pchunk = _prefix_chunk(step.batch, step.num_kv_heads, step.max_context_len, step.block_size)
     assert tiles == -(-1024 // pchunk) * (((members + 63) // 64 + 1) // 2)
 
 
@@ -147,7 +148,7 @@ def test_shared_prefix_shapes(cuda_device, lens, hq, hkv, d, bs, nshared, nblk, 
     (groups, members, tiles), _, _ = _run(step, cuda_device, store=store, min_group=4)
     assert (groups, members) == (1, nshared)
     tq = 128 // (hq // hkv if (hq // hkv) & (hq // hkv - 1) == 0 else 1)
-    pchunk = _prefix_chunk(step.batch, hkv, step.max_context_len)
+    pchunk = _prefix_chunk(step.batch, hkv, step.max_context_len, step.block_size)
     assert tiles == -(-nblk * bs // pchunk) * ((-(-nshared // tq) + 1) // 2)   # query-tile pairs
 
 
@@ -159,7 +160,7 @@ def test_prefix_partitions_of_two_key_tiles(cuda_device):
     share = np.array([i % 4 != 3 for i in range(16)])
     step = make_decode_step(33, lens, num_q_heads=16, num_kv_heads=8, head_dim=128,
                             block_size=64, shared_prefix_blocks=8, share=share)
-    pchunk = _prefix_chunk(step.batch, 8, step.max_context_len)
+    pchunk = _prefix_chunk(step.batch, 8, step.max_context_len, step.block_size)
     assert pchunk == 256
     (groups, members, tiles), _, _ = _run(step, cuda_device, min_group=4)
     assert (groups, members) == (1, 12)
@@ -179,7 +180,7 @@ def test_two_groups_and_a_short_common_run(cuda_device):
     (groups, members, tiles), _, _ = _run(step, cuda_device, min_group=4)
     assert (groups, members) == (2, 20)
     # one query tile (pair) per group; prefixes of 160 and 64 keys in partitions of pchunk
-    pchunk = _prefix_chunk(step.batch, 2, step.max_context_len)
+    pchunk = _prefix_chunk(step.batch, 2, step.max_context_len, step.block_size)
     assert tiles == -(-160 // pchunk) + -(-64 // pchunk)
 
 
