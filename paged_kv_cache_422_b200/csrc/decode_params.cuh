@@ -54,6 +54,11 @@ struct AttnParams {
     int32_t* group_start;          // [groups + 1]
     int32_t* group_len;            // [groups] prefix tokens
     int min_members, pchunk, ptq;  // smallest group, prefix keys per partition, members per tile
+    // 1 when the grid launched just before the worker is the shared-prefix tile kernel: that
+    // kernel lets the worker launch only once the plan has completed, so the worker starts at
+    // once, runs beside the prefix tiles, and waits for their grid at its end (a kernel after
+    // the worker then sees both grids' partials)
+    int wait_at_end;
 };
 
 template <int D, int GMAX>

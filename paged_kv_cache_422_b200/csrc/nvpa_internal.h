@@ -83,7 +83,7 @@ struct DecodePrefixArgs {
     float* lse_part;
     int s_max, pchunk;
     long long max_entries;       // host bound on the number of tile entries
-    int max_ctas;                // grid cap (0: two per SM)
+    int max_ctas;                // grid cap (0: one per SM)
     bool pdl;                    // launch as a programmatic dependent of the previous kernel
 };
 // Query heads that share one 128-row tensor-core tile (the group size when it is a power

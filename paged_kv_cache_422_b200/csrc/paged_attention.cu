@@ -116,7 +116,9 @@ paged_attention_kernel(const AttnParams p) {
     int it_ntiles = 0, it_t = 0, it_fb = 0, it_blk = -1;
     const int32_t* it_bt = nullptr;
 
-    pdl_wait();   // the plan (and everything before it on the stream) has completed
+    // the plan (and everything before it on the stream) has completed after this wait; with
+    // wait_at_end the grid before this one only let it launch once that was so
+    if (!p.wait_at_end) pdl_wait();
     // Lane 0 holds the next item index, requested one item ahead.
     const int total_items = __ldcg(p.counter + 1);
     int nx_item = 0;
@@ -304,6 +306,7 @@ paged_attention_kernel(const AttnParams p) {
     }
     cp_async_wait<0>();
     pdl_launch_dependents();
+    if (p.wait_at_end) pdl_wait();   // the shared-prefix tiles' grid has completed
 }
 
 // ------------------------------------------------------------------------------------
@@ -559,6 +562,7 @@ nvpa_status_t run_paged_decode(const DecodeCall& c, cudaStream_t stream) {
         e = launch_decode_prefix_tcgen05(a, stream);
         if (e != cudaSuccess) return cuda_failure(e, "decode shared-prefix launch");
         count_launches(1);
+        p.wait_at_end = 1;   // the worker runs beside the prefix tiles
     } else {
         decode_plan_kernel<<<1, 1024, 0, stream>>>(p);
         e = cudaGetLastError();

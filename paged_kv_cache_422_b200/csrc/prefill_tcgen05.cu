@@ -962,6 +962,10 @@ prefill_tcgen05_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_c
 //               warps of a row exchange its largest score and, at the end, its sum through
 //               shared memory; each warp also stores its half of the row's Q into TMEM.
 constexpr int kStages2 = 6;
+// Units (query tiles) per CTA below which the prefix grid leaves CTAs idle: with about
+// three units each the tiles of a decode step's shared prefixes take a fifth of the SMs or
+// less, and the split-KV worker, which runs beside them, streams on the rest.
+constexpr int kPrefixUnitsPerCta = 3;
 constexpr uint32_t kS2Cols = 128, kO2Col = 256, kQ2Col = 384;
 
 template <int D>
@@ -1000,8 +1004,6 @@ prefix_tiles_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_cons
     UnitDesc* unit_ring = reinterpret_cast<UnitDesc*>(smem + L::RING_OFF);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // let the decode worker's CTAs launch as this grid's CTAs finish
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) {
         for (int b = 0; b < 2; ++b) {
             mbar_init(bars + L::B_SFULL + b, 1);
@@ -1037,9 +1039,17 @@ prefix_tiles_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_cons
     // launched as a programmatic dependent of the decode plan: nothing the plan writes is
     // read before this wait
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // The decode worker may launch once every CTA of this grid is past that wait: it reads
+    // the plan's tables without a wait of its own and runs on the SMs this grid leaves free
+    // (most CTAs find no tile and exit at once), then waits for this grid at its end.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     // one unit per query tile: the two tiles of a plan entry, for every head group
     const int total = __ldcg(p.ntiles) * p.hgroups * 2;
+    // Only the first ceil(total / kPrefixUnitsPerCta) CTAs take units (every CTA when there
+    // are more units than that per CTA); the others exit at once and leave their SMs to the
+    // HBM-bound worker running beside this grid.
+    const bool idle_cta = (long long)blockIdx.x * kPrefixUnitsPerCta >= (long long)total;
     auto unit_of = [&](int idx, int4& e, int& hg) {
         hg = idx % p.hgroups;
         const int4 pe = __ldg(p.tiles + idx / (2 * p.hgroups));
@@ -1071,7 +1081,9 @@ prefix_tiles_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_cons
             const int npieces = (min(kKV, lk - key0) + piece - 1) / piece;
             return lane < npieces ? __ldg(bt + ((kbeg + key0 + lane * piece) >> p.block_shift)) : kNoPiece;
         };
-        auto claim_next = [&]() -> int { return lane == 0 ? atomicAdd(p.unit_counter, 1) : 0; };
+        auto claim_next = [&]() -> int {
+            return lane == 0 ? (idle_cta ? total : atomicAdd(p.unit_counter, 1)) : 0;
+        };
         auto resolve = [&](int pending) -> int {
             const int i = __shfl_sync(0xffffffffu, pending, 0);
             return i < total ? i : -1;

@@ -168,6 +168,24 @@ def test_prefix_partitions_of_two_key_tiles(cuda_device):
     assert tiles == 2
 
 
+def test_prefix_units_beyond_three_per_sm(cuda_device):
+    """512 sequences that all share a 3072-token prefix: 8 query tiles of 64 members, 8
+    prefix partitions of 384 keys and 8 head groups make 512 single-tile units, more than
+    three for each CTA of the one-per-SM prefix grid, so every CTA takes units (at batch
+    512 with a 1024-token prefix only the first 32 do and the worker streams on the other
+    SMs).  Both pools bit-exact; 47 sampled sequences against the oracle."""
+    lens = [3073 + (7 * i) % 227 for i in range(512)]
+    step = make_decode_step(35, lens, num_q_heads=16, num_kv_heads=8, head_dim=128,
+                            block_size=256, num_blocks=600, shared_prefix_blocks=12,
+                            share=np.ones(512, bool))
+    pchunk = _prefix_chunk(step.batch, 8, step.max_context_len, step.block_size)
+    assert pchunk == 384
+    (groups, members, tiles), _, _ = _run(step, cuda_device, seqs=list(range(0, 512, 11)))
+    assert (groups, members) == (1, 512)
+    assert tiles == (3072 // pchunk) * (512 // 64 // 2)
+    assert tiles * 8 * 2 > 3 * 148
+
+
 def test_two_groups_and_a_short_common_run(cuda_device):
     """Two groups with different donors; one member of the second group shares only two
     of the donor's four blocks, so that group's prefix is two blocks."""
