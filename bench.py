@@ -563,6 +563,16 @@ def end_to_end(run_step, packed, out, stream, steps, warmup, dev):
     return ms, br, out_host.numel() * out_host.element_size()
 
 
+# Queued on the step stream ahead of the start event (about 1 ms at 1.9 GHz): the host
+# enqueues the first steps while the GPU still runs it, so the region does not begin with
+# an idle GPU waiting for the first step's launches.  Without it the first of the timed
+# steps measured 56-130 us longer than the others on the decode workloads: the host's time
+# to enqueue one step.
+LEAD_SLEEP_CYCLES = 2_000_000
+TIMING = ("CUDA events on the step stream; a ~1 ms sleep kernel queued before the start event "
+          "(after the barrier and synchronize) so that the host enqueues ahead of the GPU")
+
+
 def timed_steps(step_fn, steps, stream, flush, dev):
     """Run `steps` steps on `stream`, each bracketed by CUDA events; with `flush`, L2 is
     evicted before every step, outside its events.  Returns (total ms of the region, list of
@@ -571,6 +581,8 @@ def timed_steps(step_fn, steps, stream, flush, dev):
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(LEAD_SLEEP_CYCLES)
     start.record(stream)
     for i in range(steps):
         if flush is not None:
@@ -636,13 +648,17 @@ def run_nvpa(args) -> int:
         if ev is not None:
             ev[1].record(stream)
 
+    # the warm-up steps run as the timed ones do (flush included), so that the first timed
+    # flush and step are not the first to touch the flush buffer or its kernels
+    flush = make_l2_flush(dev, args.flush_l2)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
+            if flush is not None:
+                flush(stream)
             one_step()
     torch.cuda.synchronize(dev)
 
     # ---------------- timed region: K steps, device-timed ----------------
-    flush = make_l2_flush(dev, args.flush_l2)
     with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
         barrier(dev)
         torch.cuda.synchronize(dev)
@@ -688,6 +704,7 @@ def run_nvpa(args) -> int:
                     total_context_tokens=int(step.context_lens.sum()),
                     unique_kv_bytes=work["kv_unique"], step_bytes=work["step"],
                     parallelism=f"replicas x{world}" if world > 1 else "single GPU",
+                    timing=TIMING,
                     l2=(L2_FLUSHED + "; %.3f GB of unique K/V per step vs 126 MB L2"
                         % (work["kv_unique"] / 1e9))
                        if args.flush_l2 else
@@ -750,11 +767,13 @@ def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
         if ev is not None:
             ev[1].record(stream)
 
+    flush = make_l2_flush(dev, args.flush_l2)   # warm-up as the timed steps, flush included
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
+            if flush is not None:
+                flush(stream)
             one_step()
     torch.cuda.synchronize(dev)
-    flush = make_l2_flush(dev, args.flush_l2)
 
     step_evs = []
 
@@ -805,6 +824,7 @@ def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
                     num_q_heads=step.num_q_heads, num_kv_heads=step.num_kv_heads,
                     head_dim=step.head_dim, block_size=step.block_size,
                     algorithmic_tflop=work["flops"] / 1e12,
+                    timing=TIMING,
                     l2=(L2_FLUSHED
                         if args.flush_l2 else
                         "inputs larger than L2, not flushed: each step stores 101 MB of new K/V "
