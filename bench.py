@@ -505,7 +505,9 @@ def end_to_end(run_step, packed, out, stream, steps, warmup, dev):
     one stream, kernels on `stream`, read-backs on a third; step i + 1's upload and step
     i - 1's read-back run while step i computes.  A buffer is reused only after the step
     that used it two steps earlier is done with it.  The timed region starts before the
-    first upload and ends after the last read-back.  `run_step(inputs, out)` enqueues one
+    first upload (behind the same lead sleep as the device-timed steps, so that the host
+    enqueues ahead of the GPU) and ends after the last read-back; the first upload and
+    the last read-back, which nothing overlaps, are inside it.  `run_step(inputs, out)` enqueues one
     step on `stream`.  Returns (ms per step, breakdown of medians: h2d, compute, d2h in
     device ms and host ms spent enqueueing a step, d2h bytes per step)."""
     import torch
@@ -544,6 +546,8 @@ def end_to_end(run_step, packed, out, stream, steps, warmup, dev):
     barrier(dev)
     hist = []
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(LEAD_SLEEP_CYCLES)
     e0.record(stream)
     up.wait_event(e0)
     host_s = []
@@ -563,14 +567,17 @@ def end_to_end(run_step, packed, out, stream, steps, warmup, dev):
     return ms, br, out_host.numel() * out_host.element_size()
 
 
-# Queued on the step stream ahead of the start event (about 1 ms at 1.9 GHz): the host
-# enqueues the first steps while the GPU still runs it, so the region does not begin with
+# Queued on the step stream ahead of the start event (about 0.2 ms at 1.9 GHz): the host
+# enqueues the first step while the GPU still runs it, so the region does not begin with
 # an idle GPU waiting for the first step's launches.  Without it the first of the timed
 # steps measured 56-130 us longer than the others on the decode workloads: the host's time
-# to enqueue one step.
-LEAD_SLEEP_CYCLES = 2_000_000
-TIMING = ("CUDA events on the step stream; a ~1 ms sleep kernel queued before the start event "
-          "(after the barrier and synchronize) so that the host enqueues ahead of the GPU")
+# to enqueue one step (about 0.1 ms).  It is kept that short so that a host-bound run (the
+# tiny batch, whose steps take less GPU time than their enqueueing) hides at most about
+# two steps of host time.
+LEAD_SLEEP_CYCLES = 400_000
+TIMING = ("CUDA events on the step stream; a ~0.2 ms sleep kernel queued before the start event "
+          "(after the barrier and synchronize) so that the first step's launches are queued "
+          "before the GPU reaches them")
 
 
 def timed_steps(step_fn, steps, stream, flush, dev):
