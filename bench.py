@@ -492,8 +492,9 @@ class PackedInputs:
 
 
 E2E_COPIES = ("every step: one packed host-to-device copy of all its inputs from pinned memory and "
-              "a device-to-host copy of its output, both inside the timed region; double-buffered "
-              "so that step i+1's upload and step i-1's read-back overlap step i's kernels")
+              "a device-to-host copy of its output, both inside the timed region; triple-buffered "
+              "so that the next steps' uploads and the previous step's read-back overlap step i's "
+              "kernels")
 
 
 def end_to_end(run_step, packed, out, stream, steps, warmup, dev):
@@ -501,18 +502,21 @@ def end_to_end(run_step, packed, out, stream, steps, warmup, dev):
     copies all of its inputs from pinned host memory (one packed host-to-device copy),
     runs on the device copies, and copies its output back to pinned host memory.
     Consecutive steps are independent batches, so the copies are pipelined the way a
-    serving loop prefetches: two device input buffers and two output buffers, uploads on
-    one stream, kernels on `stream`, read-backs on a third; step i + 1's upload and step
-    i - 1's read-back run while step i computes.  A buffer is reused only after the step
-    that used it two steps earlier is done with it.  The timed region starts before the
+    serving loop prefetches: three device input buffers and three output buffers, uploads
+    on one stream, kernels on `stream`, read-backs on a third; the uploads of the next
+    steps and the read-back of the last one run while step i computes.  A buffer is reused
+    only after the step that used it three steps earlier is done with it (with two, an
+    upload as long as a step, as on hosts whose small pinned copies run at 14 GB/s, left
+    no slack).  The timed region starts before the
     first upload (behind the same lead sleep as the device-timed steps, so that the host
     enqueues ahead of the GPU) and ends after the last read-back; the first upload and
     the last read-back, which nothing overlaps, are inside it.  `run_step(inputs, out)` enqueues one
     step on `stream`.  Returns (ms per step, breakdown of medians: h2d, compute, d2h in
     device ms and host ms spent enqueueing a step, d2h bytes per step)."""
     import torch
-    packs = [packed, packed.twin()]
-    outs = [out, torch.empty_like(out)]
+    nbuf = 3
+    packs = [packed] + [packed.twin() for _ in range(nbuf - 1)]
+    outs = [out] + [torch.empty_like(out) for _ in range(nbuf - 1)]
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     up = torch.cuda.Stream(device=dev)
     down = torch.cuda.Stream(device=dev)
@@ -520,15 +524,15 @@ def end_to_end(run_step, packed, out, stream, steps, warmup, dev):
 
     # ev: 0/1 upload start/end (up), 2/3 compute start/end (stream), 4/5 read-back (down)
     def one(i, ev, hist):
-        b = i & 1
-        if i >= 2:
-            up.wait_event(hist[i - 2][3])       # step i - 2 has finished reading this input buffer
+        b = i % nbuf
+        if i >= nbuf:
+            up.wait_event(hist[i - nbuf][3])     # that step has finished reading this input buffer
         ev[0].record(up)
         packs[b].upload(up)
         ev[1].record(up)
         stream.wait_event(ev[1])
-        if i >= 2:
-            stream.wait_event(hist[i - 2][5])   # step i - 2's read-back is done with this output
+        if i >= nbuf:
+            stream.wait_event(hist[i - nbuf][5])  # that step's read-back is done with this output
         ev[2].record(stream)
         run_step(packs[b].views, outs[b])
         ev[3].record(stream)
@@ -539,7 +543,7 @@ def end_to_end(run_step, packed, out, stream, steps, warmup, dev):
         ev[5].record(down)
 
     hist = []
-    for i in range(max(2, warmup)):
+    for i in range(max(nbuf, warmup)):
         hist.append(mk())
         one(i, hist[-1], hist)
     torch.cuda.synchronize(dev)
@@ -860,8 +864,10 @@ def run_nvpa_prefill(args, step, dev, lib, world, rank) -> int:
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description="paged-KV attention benchmark (one JSON line)")
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    # 10 warm-up launches and 100 timed steps by default (the median of 100 iterations):
+    # about 30 ms of timed work at the default workload
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["nvpa", "reference"], default="nvpa")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--num-splits", type=int, default=0)
