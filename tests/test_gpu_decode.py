@@ -86,6 +86,21 @@ def test_decode_b512_shared_prefix_sampled(cuda_device):
     assert len(step.shared_blocks) == 4 and shared.sum() == 256
 
 
+def test_decode_many_rows_head_dim_64(cuda_device):
+    """1600 sequences x 4 query heads (6400 rows, head_dim 64) with 700-900 keys each: every
+    row has two or three 352-key partitions, more rows than the combine's CTAs cover in one
+    wave of residents (one warp per row)."""
+    lens = [700 + (37 * i) % 201 for i in range(1600)]
+    step = make_decode_step(17, lens, num_q_heads=4, num_kv_heads=2, head_dim=64, block_size=16)
+    kc, vc, bad = oracle_after_store(step)
+    assert bad == []
+    t = decode_to_device(step, cuda_device)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    out, lse = _run(step, t, err=err)
+    assert err.item() == 0
+    _check(step, kc, vc, out, lse, list(range(0, 1600, 53)) + [1599], "1600 x 4 rows, head_dim 64")
+
+
 def test_decode_long_context_block16(cuda_device):
     step, kc, vc = _workload("decode_long_b8_ctx32k_bs16")
     t = decode_to_device(step, cuda_device)

@@ -87,6 +87,27 @@ def test_split_kv_long_context_workload(cuda_device):
     assert_attention_close(out[seqs], ref, "long-context split-KV")
 
 
+def test_partial_fp32_output_at_batch_512(cuda_device):
+    """The partial entry point (fp32 output and lse) on the batch-512 workload: 8192 rows of
+    several partitions each, more than the combine's CTAs cover in one wave; sampled
+    sequences against the oracle."""
+    step = _stored(WORKLOADS["decode_b512_shared_prefix"]())
+    t = decode_to_device(step, cuda_device)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    o, lse = nvpa.paged_decode_partial(t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                                       t["context_lens"], step.max_context_len, step.scale,
+                                       err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    seqs = list(range(0, 512, 29)) + [int(np.argmax(step.context_lens))]
+    ref, ref_lse = oracle.paged_decode_attention(step.q[seqs], step.k_pool, step.v_pool,
+                                                 step.block_tables[seqs], step.context_lens[seqs],
+                                                 step.scale)
+    sel = torch.as_tensor(seqs, device=cuda_device)
+    assert np.max(np.abs(o[sel].cpu().numpy() - ref)) < 2e-3
+    assert_lse_close(lse[sel], ref_lse, "batch-512 partial lse")
+
+
 def test_lse_combine_weights_and_empty_rows(cuda_device):
     """Closed forms: equal lse -> plain mean of the parts; a -inf part weighs nothing; a
     row of -inf parts gives 0 and -inf."""
