@@ -18,7 +18,7 @@ constexpr int kCombineLoads = 8;
 constexpr int kCombineWarps = 8;   // warps per CTA
 
 template <int D, int W>
-__global__ void __launch_bounds__(kCombineWarps * 32) decode_combine_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(kCombineWarps * 32, 4) decode_combine_kernel(const AttnParams p) {
     constexpr int DPL = D / 32;   // output dims per lane
     constexpr int R = kCombineWarps / W;   // rows per CTA
     __shared__ float red[kCombineWarps][D];
@@ -29,6 +29,10 @@ __global__ void __launch_bounds__(kCombineWarps * 32) decode_combine_kernel(cons
     const int part = warp % W;                 // this warp's share of the row's partitions
     const bool row_ok = w < p.batch * p.hq;
     const int b = row_ok ? w / p.hq : 0;
+    const float* lp = p.lse_part + (size_t)(row_ok ? w : 0) * p.s_max;
+    // the row's first 32 lse slots are read together with its partition count (slots past
+    // the count hold stale values and are dropped below), saving a dependent round of loads
+    const float lse0 = (row_ok && lane < p.s_max) ? __ldcg(lp + lane) : -INFINITY;
     const int ns = row_ok ? __ldcg(p.nsplit + b) : 0;
     // (no early return: the shares of a row meet at the barrier below)
     const bool merge = ns > 1;
@@ -37,15 +41,18 @@ __global__ void __launch_bounds__(kCombineWarps * 32) decode_combine_kernel(cons
     for (int k = 0; k < DPL; ++k) acc[k] = 0.f;
     float tot = 0.f, mx = -INFINITY;
     if (merge) {
-        const float* lp = p.lse_part + (size_t)w * p.s_max;
         const float* op = p.o_part + (size_t)w * p.s_max * D + lane * DPL;
-        for (int s = lane; s < ns; s += 32) mx = fmaxf(mx, __ldcg(lp + s));
+        mx = lane < ns ? lse0 : -INFINITY;
+        for (int s = lane + 32; s < ns; s += 32) mx = fmaxf(mx, __ldcg(lp + s));
         mx = warp_max(mx);
         const int per = (ns + W - 1) / W;
         const int s_begin = min(ns, part * per), s_end = min(ns, s_begin + per);
         if (mx > -INFINITY) {
             for (int s0 = s_begin; s0 < s_end; s0 += 32) {
-                const float wl = (s0 + lane < s_end) ? fast_exp2((__ldcg(lp + s0 + lane) - mx) * kLog2e) : 0.f;
+                // (the shuffle runs in every lane: s0 is the same across the warp)
+                const float sh = __shfl_sync(0xffffffffu, lse0, (s0 + lane) & 31);
+                const float ls = s0 + lane < s_end ? (s0 + lane < 32 ? sh : __ldcg(lp + s0 + lane)) : -INFINITY;
+                const float wl = (s0 + lane < s_end) ? fast_exp2((ls - mx) * kLog2e) : 0.f;
                 tot += wl;
                 const int n = min(32, s_end - s0);
                 int j = 0;
