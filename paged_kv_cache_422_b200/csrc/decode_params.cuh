@@ -41,7 +41,7 @@ struct AttnParams {
     float* lse_part;
     int4* items;
     int32_t* nsplit;
-    int32_t* counter;              // [0] next item, [1] number of items
+    int32_t* counter;              // [0] items claimed after the first round, [1] number of items
     int32_t* err;
     int batch, hq, hkv, group;
     int max_blocks, num_blocks, block_size, block_shift;

@@ -19,9 +19,9 @@ namespace nvpa {
 //                                        for all members on the tensor cores;
 //   private partitions npc .. npc+nsp-1 keys [prefix + s * chunk, ...), worker items;
 // and the combine merges all npc + nsp partials.  Sequences outside a group get the plain
-// decode plan's items.  Counters in the workspace: [0] next item, [1] items, [2] groups,
-// [3] members, [4] prefix work units (pairs of query tiles of one group and partition),
-// [5] the prefix kernel's unit counter.
+// decode plan's items.  Counters in the workspace: [0] items claimed after the worker's
+// first round, [1] items, [2] groups, [3] members, [4] prefix work units (pairs of query
+// tiles of one group and partition), [5] the prefix kernel's unit counter.
 
 __global__ void __launch_bounds__(1024) decode_plan_shared_kernel(const AttnParams p) {
     extern __shared__ int sh[];

@@ -119,10 +119,13 @@ paged_attention_kernel(const AttnParams p) {
     // the plan (and everything before it on the stream) has completed after this wait; with
     // wait_at_end the grid before this one only let it launch once that was so
     if (!p.wait_at_end) pdl_wait();
-    // Lane 0 holds the next item index, requested one item ahead.
+    // A warp's first item is its index in the grid; the counter hands out the items after
+    // the first round, and lane 0 holds the next one, requested one item ahead.  (Claiming
+    // the first items from the counter as well made the warps that started first take two
+    // items each when there are about as many items as warps, and left the others idle.)
     const int total_items = __ldcg(p.counter + 1);
-    int nx_item = 0;
-    if (lane == 0) nx_item = atomicAdd(p.counter, 1);
+    const int nwarps = gridDim.x * kAttnWarps;
+    int nx_item = blockIdx.x * kAttnWarps + warp;
 
     auto load_blocks = [&]() {
         it_fb = it_k0 >> p.block_shift;
@@ -145,7 +148,7 @@ paged_attention_kernel(const AttnParams p) {
             it_valid = false;
             return;
         }
-        if (lane == 0) nx_item = atomicAdd(p.counter, 1);
+        if (lane == 0) nx_item = nwarps + atomicAdd(p.counter, 1);
         const int4 d = __ldcg(reinterpret_cast<const int4*>(p.items) + idx / p.hkv);
         it_valid = true;
         it_seq = d.x;
