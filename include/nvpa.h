@@ -402,6 +402,18 @@ nvpa_status_t nvpa_gather_kv(void* dst, const void* cache,
                              int num_kv_heads, int head_dim, int num_blocks, int block_size,
                              int32_t* err_flag, cudaStream_t stream);
 
+/*
+ * nvpa_check_bounded_wait -- test helper for the tensor-core kernels' time-bounded waits:
+ * one warp waits, with the same wait those kernels use, on a shared-memory barrier that
+ * nothing arrives at.  After 2 s the wait gives up, NVPA_FLAG_TIMEOUT is OR-ed into
+ * *err_flag and the kernel returns; the context stays usable.  (No page defines this: it
+ * shows on the device that a wait which cannot complete ends in a status, not a hang.)
+ *
+ *   err_flag        device int32, required (not null).
+ * Errors: NVPA_ERR_INVALID_ARG for a null err_flag; NVPA_ERR_CUDA if the launch fails.
+ */
+nvpa_status_t nvpa_check_bounded_wait(int32_t* err_flag, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

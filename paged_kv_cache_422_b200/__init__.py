@@ -15,6 +15,7 @@ from ._lib import (  # noqa: F401
     lib,
 )
 from .api import (  # noqa: F401
+    check_bounded_wait,
     decode_shared_prefix_workspace_size,
     decode_step,
     decode_step_shared_prefix,

@@ -55,6 +55,7 @@ SIGNATURES = {
     "nvpa_varlen_prefill_attention": (_i, [_p, _p, _p, _p, _p, _p, _i, _p, _p, _i, _i, _i, _i,
                                            _i, _i, _i, _i, _i, _f, _i, _p, _sz, _p, _p]),
     "nvpa_gather_kv": (_i, [_p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _p, _p]),
+    "nvpa_check_bounded_wait": (_i, [_p, _p]),
 }
 
 

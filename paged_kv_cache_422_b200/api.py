@@ -242,6 +242,13 @@ def varlen_prefill_attention(q, k_cache, v_cache, block_tables, cu_seqlens_q, cu
     return (out, lse) if return_lse else out
 
 
+def check_bounded_wait(err_flag, stream=None):
+    """Run the bounded-wait check kernel (a wait that cannot complete); afterwards
+    err_flag holds NVPA_FLAG_TIMEOUT."""
+    _need(err_flag, _I32, "err_flag")
+    check(lib().nvpa_check_bounded_wait(_ptr(err_flag), _stream_handle(stream)), "nvpa_check_bounded_wait")
+
+
 def gather_kv(cache, block_tables, cu_seqlens_k, total_k, out=None, err_flag=None, stream=None):
     """Contiguous copy of each sequence's paged rows: [total_k, Hkv, D] bf16."""
     _need(cache, _BF16, "cache", 4)

@@ -362,4 +362,10 @@ nvpa_status_t nvpa_gather_kv(void* dst, const void* cache, const int32_t* block_
                          num_kv_heads, head_dim, num_blocks, block_size, err_flag, stream);
 }
 
+nvpa_status_t nvpa_check_bounded_wait(int32_t* err_flag, cudaStream_t stream) {
+    g_last_error[0] = 0;
+    NVPA_REQUIRE(err_flag != nullptr, NVPA_ERR_INVALID_ARG, "err_flag must not be null");
+    return run_bounded_wait_check(err_flag, stream);
+}
+
 }  // extern "C"

@@ -113,5 +113,6 @@ nvpa_status_t run_gather_kv(void* dst, const void* cache, const int32_t* block_t
                             int max_blocks_per_seq, const int32_t* cu_seqlens_k, int batch,
                             int total_k, int hkv, int head_dim, int num_blocks, int block_size,
                             int32_t* err_flag, cudaStream_t stream);
+nvpa_status_t run_bounded_wait_check(int32_t* err_flag, cudaStream_t stream);
 
 }  // namespace nvpa

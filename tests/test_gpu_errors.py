@@ -1,13 +1,17 @@
 """Error behaviour on the GPU: host-side statuses and device-side flags (no faults)."""
 
+import time
+
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import paged_kv_cache_422_b200 as nvpa
 from paged_kv_cache_422_b200 import NvpaError
 from synth import make_decode_step, make_prefill_step
 from synth.device import decode_to_device, i32, prefill_to_device
+from tests.helpers import assert_attention_close, oracle_after_store
 
 pytestmark = pytest.mark.gpu
 
@@ -100,3 +104,37 @@ def test_prefill_bad_block_id_is_flagged_and_stays_finite(cuda_device):
                                              step.cu_seqlens_k, step.scale)
     q1 = int(step.cu_seqlens_q[1])
     assert_attention_close(out[q1:], ref[q1:], "prefill, sequence with a valid table")
+
+
+
+def test_bounded_wait_runs_out_with_a_status(cuda_device):
+    """A wait that cannot complete (a barrier nothing arrives at, waited on with the
+    tensor-core kernels' own bounded wait) gives up after about 2 s, flags
+    NVPA_FLAG_TIMEOUT and returns; the next prefill on the same context, whose kernel
+    uses the same waits, completes with no flag and matches the oracle."""
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    nvpa.check_bounded_wait(err)
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    assert err.item() == nvpa.NVPA_FLAG_TIMEOUT
+    assert 1.5 < elapsed < 60.0
+    assert nvpa.lib().nvpa_check_bounded_wait(None, None) == 1   # null err_flag: INVALID_ARG
+
+    step = make_prefill_step(300, [200, 90], cached_blocks=[1, 0], num_q_heads=8, num_kv_heads=2,
+                             head_dim=128, block_size=64)
+    t = prefill_to_device(step, cuda_device)
+    err2 = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    nvpa.store_kvcache(t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], t["slot_mapping"],
+                       err_flag=err2)
+    out = nvpa.varlen_prefill_attention(t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                                        t["cu_seqlens_q"], t["cu_seqlens_k"], step.max_seqlen_q,
+                                        step.max_seqlen_k, step.scale, err_flag=err2)
+    torch.cuda.synchronize()
+    assert err2.item() == 0
+    kc, vc, bad = oracle_after_store(step)
+    assert bad == []
+    ref, _ = oracle.varlen_prefill_attention(step.q, kc, vc, step.block_tables, step.cu_seqlens_q,
+                                             step.cu_seqlens_k, step.scale)
+    assert_attention_close(out, ref, "prefill after a timed-out wait")
