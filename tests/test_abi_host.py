@@ -149,6 +149,11 @@ def test_gather_host_checks(lib):
     assert f(None, FAKE, FAKE, 4, FAKE, 2, 10, 2, 64, 8, 16, None, None) == _lib.NVPA_ERR_INVALID_ARG
 
 
+def test_bounded_wait_check_host_checks(lib):
+    # a null error word is refused before anything is launched
+    assert lib.nvpa_check_bounded_wait(None, None) == _lib.NVPA_ERR_INVALID_ARG
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(_lib, "_lib", None)
